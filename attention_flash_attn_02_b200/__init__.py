@@ -1,0 +1,185 @@
+"""Python binding of libattn_sm100.so (B200 fused attention).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/attn.h``.  PyTorch supplies device
+memory and the current stream.  If the shared library is missing, every call
+raises -- there is no fallback.
+
+Functions mirror the C entry points:
+
+* ``attn_fwd(q, k, v, scale=None, causal=False, window=0, o=None, lse=None)``
+* ``attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, ...)``
+* ``attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, ...)``
+* ``attn_decode_workspace_bytes(B, Hq, max_pages_per_seq, D)``
+* ``attn_last_device_error()``, ``attn_status_str(code)``,
+  ``attn_set_debug(flags, wait_timeout_ns)``, ``attn_version()``
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libattn_sm100.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_CUDA = -3
+ATTN_ERR_TIMEOUT = -4
+ATTN_ERR_BOUNDS = -5
+ATTN_DEBUG_BOUNDS = 1
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what} failed: {attn_status_str(status)} ({status})")
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Loads the shared library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} not found: build it with `python -m attention_flash_attn_02_b200.build`")
+    lib = ctypes.CDLL(path)
+    c_int, c_float, c_void_p, c_size_t = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [c_void_p] * 5 + [c_int] * 6 + [c_float, c_int, c_int, c_void_p]
+    lib.attn_fwd.restype = c_int
+    lib.attn_fwd_fp8.argtypes = [c_void_p] * 5 + [c_int] * 6 + [c_float, c_int, c_int] + [c_float] * 3 + [c_void_p]
+    lib.attn_fwd_fp8.restype = c_int
+    lib.attn_decode_workspace_bytes.argtypes = [c_int] * 4
+    lib.attn_decode_workspace_bytes.restype = c_size_t
+    lib.attn_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p, c_size_t, c_void_p]
+    lib.attn_decode_paged.restype = c_int
+    lib.attn_last_device_error.argtypes = [c_void_p]
+    lib.attn_last_device_error.restype = c_int
+    lib.attn_status_str.argtypes = [c_int]
+    lib.attn_status_str.restype = ctypes.c_char_p
+    lib.attn_set_debug.argtypes = [c_int, ctypes.c_ulonglong]
+    lib.attn_set_debug.restype = c_int
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = c_int
+    _lib = lib
+    return lib
+
+
+def attn_status_str(status: int) -> str:
+    return load().attn_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _stream_handle(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None and t.numel() > 0 else ctypes.c_void_p(0)
+
+
+def attn_fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, window: int = 0,
+             o=None, lse=None, stream=None):
+    """bf16 attention forward.  q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D], contiguous,
+    on the GPU.  Returns (o bf16 [B,Hq,Lq,D], lse fp32 [B,Hq,Lq])."""
+    import torch
+    lib = load()
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Hq, Lq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    for t in (q, k, v, o, lse):
+        if not t.is_contiguous():
+            raise ValueError("attn_fwd: tensors must be contiguous")
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("attn_fwd: q, k, v must be bfloat16")
+    st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
+                      float(scale), int(bool(causal)), int(window), _stream_handle(stream))
+    _check(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float,
+                 scale: Optional[float] = None, causal: bool = False, window: int = 0,
+                 o=None, lse=None, stream=None):
+    """e4m3 attention forward (bf16 output); tensors torch.float8_e4m3fn."""
+    import torch
+    lib = load()
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Hq, Lq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn or not t.is_contiguous():
+            raise TypeError("attn_fwd_fp8: q, k, v must be contiguous float8_e4m3fn")
+    st = lib.attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
+                          float(scale), int(bool(causal)), int(window), float(q_descale),
+                          float(k_descale), float(v_descale), _stream_handle(stream))
+    _check(st, "attn_fwd_fp8")
+    return o, lse
+
+
+def attn_decode_workspace_bytes(B: int, Hq: int, max_pages_per_seq: int, D: int) -> int:
+    return int(load().attn_decode_workspace_bytes(B, Hq, max_pages_per_seq, D))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,
+                      o=None, lse=None, workspace=None, stream=None):
+    """Single-token paged decode.  q [B,Hq,D] bf16; pools [P,16,Hkv,D] bf16;
+    block_table [B,max_pages] int32; seq_lens [B] int32; all on the GPU.
+    Returns (o bf16 [B,Hq,D], lse fp32 [B,Hq])."""
+    import torch
+    lib = load()
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = lib.attn_decode_workspace_bytes(B, Hq, max(max_pages, 1), D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("attn_decode_paged: block_table and seq_lens must be int32")
+    st = lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                               _ptr(o), _ptr(lse), B, Hq, Hkv, D, page_size, num_pages, max_pages,
+                               float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream_handle(stream))
+    _check(st, "attn_decode_paged")
+    return o, lse
+
+
+def attn_last_device_error(stream=None) -> int:
+    return int(load().attn_last_device_error(_stream_handle(stream)))
+
+
+def attn_set_debug(flags: int, wait_timeout_ns: int = 0) -> int:
+    return int(load().attn_set_debug(int(flags), int(wait_timeout_ns)))
+
+
+def attn_version() -> int:
+    return int(load().attn_version())

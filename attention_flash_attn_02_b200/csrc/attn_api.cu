@@ -1,0 +1,163 @@
+// attn_api.cu -- the C ABI of include/attn.h: argument validation (before any
+// CUDA call), the per-device status word, debug switches, and dispatch to the
+// kernel launchers.
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "internal.h"
+
+namespace attn {
+
+// One status word per device, written by kernels (never trapped on).
+__device__ int g_status;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_sms[kMaxDevices] = {0};
+std::mutex g_mu;
+std::atomic<int> g_debug_flags{0};
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}  // namespace
+
+int* device_status_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (g_status_ptr[dev]) return g_status_ptr[dev];
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  return g_status_ptr[dev];
+}
+
+int debug_flags() { return g_debug_flags.load(); }
+unsigned long long wait_timeout_ns() { return g_timeout_ns.load(); }
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+namespace {
+
+int validate_prefill(const void* q, const void* k, const void* v, void* o, const float* lse, int B, int Hq,
+                     int Hkv, int Lq, int Lk, int D, float scale, int causal, int window) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || D <= 0) return ATTN_ERR_INVALID;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
+  if (window > 0 && !causal) return ATTN_ERR_INVALID;
+  if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;  // NaN or non-positive
+  const long long nq = (long long)B * Hq * Lq;
+  const long long nk = (long long)B * Hkv * Lk;
+  if (nq > 0 && (!q || !o || !aligned16(q) || !aligned16(o))) return ATTN_ERR_INVALID;
+  if (nq > 0 && lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID;
+  if (nk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID;
+  if (B > 65535 || (long long)B * Hq > (1ll << 31) - 1 || Lq > (1 << 30) || Lk > (1 << 30))
+    return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                      int Lq, int Lk, int D, float scale, int causal, int window, attn_stream_t stream) {
+  int st = validate_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * Lq == 0) return ATTN_OK;
+  PrefillArgs a{q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, window > 0 ? window : 0, false, 1.f, 1.f, 1.f};
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                          int Hkv, int Lq, int Lk, int D, float scale, int causal, int window, float q_descale,
+                          float k_descale, float v_descale, attn_stream_t stream) {
+  int st = validate_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (!(q_descale > 0.f) || !(k_descale > 0.f) || !(v_descale > 0.f)) return ATTN_ERR_INVALID;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * Lq == 0) return ATTN_OK;
+  PrefillArgs a{q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, window > 0 ? window : 0, true,
+                q_descale, k_descale, v_descale};
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D) {
+  if (B <= 0 || Hq <= 0 || max_pages_per_seq <= 0 || D <= 0) return 0;
+  // normalised partial outputs (D floats) and their log-sum-exp (1 float)
+  return (size_t)B * Hq * decode_max_splits(max_pages_per_seq) * (size_t)(D + 1) * sizeof(float);
+}
+
+ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                               const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                               int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                               size_t workspace_bytes, attn_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages_per_seq < 0)
+    return ATTN_ERR_INVALID;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
+  if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;
+  if (B == 0) return ATTN_OK;
+  if (!q || !o || !seq_lens || !aligned16(q) || !aligned16(o)) return ATTN_ERR_INVALID;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID;
+  if (max_pages_per_seq > 0 && (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u)))
+    return ATTN_ERR_INVALID;
+  if (num_pages > 0 && (!k_pages || !v_pages || !aligned16(k_pages) || !aligned16(v_pages)))
+    return ATTN_ERR_INVALID;
+  if (D != 128 || page_size != 16 || Hq / Hkv > 32) return ATTN_ERR_UNSUPPORTED;
+  const int mp = max_pages_per_seq > 0 ? max_pages_per_seq : 1;
+  const size_t need = attn_decode_workspace_bytes(B, Hq, mp, D);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_INVALID;
+  DecodeArgs a{q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size, num_pages,
+               max_pages_per_seq, scale, workspace, workspace_bytes};
+  return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+ATTN_API int attn_last_device_error(attn_stream_t stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int* p = device_status_word();
+  if (!p) return ATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return v;
+}
+
+ATTN_API const char* attn_status_str(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID: return "ATTN_ERR_INVALID";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_BOUNDS: return "ATTN_ERR_BOUNDS";
+    default: return "ATTN_UNKNOWN_STATUS";
+  }
+}
+
+ATTN_API int attn_set_debug(int flags, unsigned long long wait_timeout_ns) {
+  const int prev = g_debug_flags.exchange(flags);
+  g_timeout_ns.store(wait_timeout_ns ? wait_timeout_ns : 2000000000ull);
+  return prev;
+}
+
+ATTN_API int attn_version(void) { return 1; }

@@ -1,0 +1,56 @@
+// internal.h -- declarations shared by the library's translation units (not
+// part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace attn {
+
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Lq, Lk, D;
+  float scale;
+  int causal, window;
+  bool fp8;
+  float q_descale, k_descale, v_descale;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_pages;
+  const void* v_pages;
+  const int* block_table;
+  const int* seq_lens;
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, D, page_size, num_pages, max_pages;
+  float scale;
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+// Device status word of the current device (nullptr on failure).
+int* device_status_word();
+// Current debug flags / wait limit (set by attn_set_debug).
+int debug_flags();
+unsigned long long wait_timeout_ns();
+// Number of SMs of the current device (cached).
+int sm_count();
+
+// Launchers: return a status code of include/attn.h.
+int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Decode work split (shared by the workspace-size query and the launcher).
+constexpr int kDecodePagesPerSplit = 32;  // 512 tokens per split CTA
+inline int decode_max_splits(int max_pages) {
+  return (max_pages + kDecodePagesPerSplit - 1) / kDecodePagesPerSplit;
+}
+
+}  // namespace attn

@@ -1,0 +1,582 @@
+// prefill_sm100.cu -- fused attention forward for B200 (sm_100a).
+//
+// Computes O = softmax(scale * Q K^T + mask) V and the per-row LSE with the
+// online-softmax recurrence of the tiled FlashAttention loop (page
+// "003-注意力机制详解：从基础Attention到DeepSeek的优化策略", §二): per K/V
+// block, S = Q K^T, new running max, rescale of the accumulator and of the
+// running sum, P = exp(S - max), acc += P V, sum += rowsum(P); at the end
+// O = acc / sum.  Scores and the accumulator never leave the SM (the "tiles
+// in SRAM, one fused kernel" design of the tqpw.cn article §4.1-4.2), and K/V
+// blocks wholly above the causal diagonal or before the sliding window are
+// never loaded (kler.cn page §一.2; window of the zeeklog page).
+//
+// B200 mapping (one persistent CTA per SM, 320 threads):
+//   warps 0-3   softmax warpgroup for Q tile 0 (one thread per query row)
+//   warps 4-7   softmax warpgroup for Q tile 1
+//   warp  8     TMA producer: Q tiles, then K_j, V_j into a ring of stages
+//   warp  9     MMA issuer (one thread) + TMEM owner
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,..).
+// P (bf16 or e4m3) is written back over the first columns of its S buffer
+// and consumed from TMEM as the A operand of O += P V.
+// The two Q tiles of a work unit share every K/V tile: for GQA they are two
+// query heads of one K/V group at the same rows; otherwise two consecutive
+// 128-row blocks of one head.  While one warpgroup runs the softmax of its
+// tile, the tensor core works on the other tile.
+//
+// Deviations from the pages' sketch: exp2 with scale*log2(e) folded in (same
+// value), and the running max is only moved when it grows by more than 8
+// (log2 units); with a stale max P stays <= 2^8, and the final O / sum and
+// LSE = max + log2(sum) are unchanged mathematically.  This removes most of
+// the accumulator rescales.
+#include <cfloat>
+#include <climits>
+#include <cstdio>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per K/V block
+constexpr int kThreads = 320;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D, bool FP8>
+struct Cfg {
+  static constexpr int EL = FP8 ? 1 : 2;                 // bytes per element
+  static constexpr int ROW_BYTES = D * EL;
+  static constexpr int NBOX = ROW_BYTES / 128;           // 128-byte swizzle columns per tile
+  static constexpr int BOX_ELEMS = 128 / EL;             // elements per box row
+  static constexpr int BOX_BYTES = kBM * 128;            // one box: 128 rows x 128 B
+  static constexpr int TILE_BYTES = kBM * ROW_BYTES;
+  static constexpr int NS = TILE_BYTES >= 32768 ? 4 : 8;  // K/V ring stages
+  static constexpr int MMA_K = FP8 ? 32 : 16;
+  static constexpr int S_KSTEPS = D / MMA_K;
+  static constexpr int PV_KSTEPS = kBN / MMA_K;
+  static constexpr int P_COLS = kBN * EL / 4;             // TMEM columns holding P
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+  static constexpr uint32_t IDESC_S = make_idesc(FP8 ? 0u : 1u, kBM, kBN, false);
+  static constexpr uint32_t IDESC_PV = make_idesc(FP8 ? 0u : 1u, kBM, D, true);
+  // shared memory: [Q0][Q1][stage 0..NS-1] (1024-aligned) + barriers
+  static constexpr int SMEM_TILES = (2 + NS) * TILE_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align slack*/ + 256 /*barriers*/;
+  static_assert(NBOX >= 1 && ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle rows");
+  static_assert(TM_O1 + D <= 512, "TMEM budget");
+};
+
+struct Params {
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Lq, Lk;
+  int group;        // Hq / Hkv
+  int pair_heads;   // 1: the two tiles are heads 2p, 2p+1 of one group
+  int n_pairs;      // units per row group
+  int n_mgroups;    // row groups
+  int n_units;
+  int causal, window;
+  float scale_log2;  // logit scale * log2(e) (fp8: times both descales)
+  float out_scale;   // 1 (bf16) or v_descale (fp8)
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+struct Unit {
+  int bh[2];  // b * Hq + head of each tile
+  int m0[2];  // first query row of each tile
+  int kvbh;   // b * Hkv + kv head
+  int kb_lo;  // first K/V block
+  int nb;     // number of K/V blocks (0: nothing visible)
+};
+
+// Visible keys [lo, hi) of query row i (bottom-right causal alignment; window
+// of W keys including the query's own position).
+__device__ __forceinline__ void key_range(int i, const Params& p, int& lo, int& hi) {
+  if (!p.causal) {
+    lo = 0;
+    hi = p.Lk;
+    return;
+  }
+  int h = i + (p.Lk - p.Lq) + 1;
+  h = h < 0 ? 0 : (h > p.Lk ? p.Lk : h);
+  hi = h;
+  lo = (p.window > 0 && h - p.window > 0) ? h - p.window : 0;
+}
+
+// Units are numbered so that the longest (latest rows under a causal mask)
+// come first; CTA c takes units c, c + grid, ...
+__device__ __forceinline__ Unit get_unit(int u, const Params& p) {
+  Unit w;
+  const int mg = p.n_mgroups - 1 - u / p.n_pairs;
+  const int pr = u % p.n_pairs;
+  if (p.pair_heads) {
+    const int hp_per_b = p.Hq >> 1;
+    const int b = pr / hp_per_b, hp = pr % hp_per_b;
+    w.bh[0] = b * p.Hq + 2 * hp;
+    w.bh[1] = w.bh[0] + 1;
+    w.m0[0] = w.m0[1] = mg * kBM;
+    w.kvbh = b * p.Hkv + (2 * hp) / p.group;
+  } else {
+    const int b = pr / p.Hq, h = pr % p.Hq;
+    w.bh[0] = w.bh[1] = b * p.Hq + h;
+    w.m0[0] = mg * 2 * kBM;
+    w.m0[1] = w.m0[0] + kBM;
+    w.kvbh = b * p.Hkv + h / p.group;
+  }
+  int lo = INT_MAX, hi = 0;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (w.m0[t] < p.Lq) {
+      const int r_last = min(w.m0[t] + kBM - 1, p.Lq - 1);
+      int lo0, hi0, lo1, hi1;
+      key_range(w.m0[t], p, lo0, hi0);
+      key_range(r_last, p, lo1, hi1);
+      if (hi1 > lo0) {  // lo and hi are non-decreasing in the row index
+        lo = min(lo, lo0);
+        hi = max(hi, hi1);
+      }
+    }
+  }
+  if (hi <= lo) {
+    w.kb_lo = 0;
+    w.nb = 0;
+  } else {
+    w.kb_lo = lo / kBN;
+    w.nb = (hi + kBN - 1) / kBN - w.kb_lo;
+  }
+  return w;
+}
+
+struct Smem {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full[2], o_empty[2];
+  uint64_t drain;
+  uint64_t kv_full[8], kv_empty[8];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<D, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t tiles_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* tiles_ptr = smem_raw + (tiles_addr - raw_addr);
+  Smem& sm = *reinterpret_cast<Smem*>(tiles_ptr + C::SMEM_TILES);
+  const uint32_t q_addr[2] = {tiles_addr, tiles_addr + (uint32_t)C::TILE_BYTES};
+  const uint32_t kv_addr0 = tiles_addr + 2u * C::TILE_BYTES;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sm.q_full[t], 1);
+      mbar_init(&sm.q_empty[t], 1);
+      mbar_init(&sm.s_full[t], 1);
+      mbar_init(&sm.p_full[t], 128);
+      mbar_init(&sm.o_full[t], 1);
+      mbar_init(&sm.o_empty[t], 128);
+    }
+    mbar_init(&sm.drain, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitGuard g{&sm.abort_flag, p.status, p.timeout_ns, true};
+  const WaitGuard g_drain{&sm.abort_flag, p.status, p.timeout_ns, false};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t seq = 0, nunit = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit w = get_unit(u, p);
+        if (w.nb <= 0) continue;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (nunit > 0) ok = mbar_wait(&sm.q_empty[t], (nunit - 1) & 1, g);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sm.q_full[t], C::TILE_BYTES);
+#pragma unroll
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_3d(q_addr[t] + bx * C::BOX_BYTES, &tm_q, &sm.q_full[t], bx * C::BOX_ELEMS, w.m0[t], w.bh[t]);
+        }
+        for (int j = 0; j < w.nb && ok; ++j) {
+          const int row = (w.kb_lo + j) * kBN;
+          for (int kind = 0; kind < 2; ++kind) {
+            const uint32_t s = seq % C::NS;
+            if (seq >= (uint32_t)C::NS) {
+              ok = mbar_wait(&sm.kv_empty[s], ((seq / C::NS) - 1) & 1, g);
+              if (!ok) break;
+            }
+            const uint32_t dst = kv_addr0 + s * C::TILE_BYTES;
+            mbar_arrive_expect_tx(&sm.kv_full[s], C::TILE_BYTES);
+            const CUtensorMap* m = kind == 0 ? &tm_k : &tm_v;
+#pragma unroll
+            for (int bx = 0; bx < C::NBOX; ++bx)
+              tma_load_3d(dst + bx * C::BOX_BYTES, m, &sm.kv_full[s], bx * C::BOX_ELEMS, row, w.kvbh);
+            ++seq;
+          }
+        }
+        ++nunit;
+      }
+      // Drain: every load this thread issued has landed before the CTA exits.
+      for (uint32_t s = 0; s < (uint32_t)C::NS && s < seq; ++s) {
+        const uint32_t last = s + ((seq - 1 - s) / C::NS) * C::NS;
+        mbar_wait(&sm.kv_full[s], (last / C::NS) & 1, g_drain);
+      }
+      if (nunit > 0)
+        for (int t = 0; t < 2; ++t) mbar_wait(&sm.q_full[t], (nunit - 1) & 1, g_drain);
+    }
+  } else if (warp == 9) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      uint32_t seq = 0, nunit = 0, pcnt[2] = {0, 0};
+      bool ok = true;
+      const uint32_t tS[2] = {tmem + C::TM_S0, tmem + C::TM_S1};
+      const uint32_t tO[2] = {tmem + C::TM_O0, tmem + C::TM_O1};
+      auto issue_s = [&](int t, uint32_t k_stage_addr) {
+#pragma unroll
+        for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
+          const uint32_t byte_k = kk * C::MMA_K * C::EL;
+          const uint32_t off = (byte_k / 128) * C::BOX_BYTES + (byte_k % 128);
+          const uint64_t a = sw128_desc(q_addr[t] + off, 16, 1024);
+          const uint64_t b = sw128_desc(k_stage_addr + off, 16, 1024);
+          if (FP8)
+            mma_f8_ss(tS[t], a, b, C::IDESC_S, kk > 0);
+          else
+            mma_f16_ss(tS[t], a, b, C::IDESC_S, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t v_stage_addr, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::PV_KSTEPS; ++kk) {
+          const uint64_t b = sw128_desc(v_stage_addr + kk * C::MMA_K * 128, C::BOX_BYTES, 1024);
+          const uint32_t a = tS[t] + kk * (C::MMA_K * C::EL / 4);
+          if (FP8)
+            mma_f8_ts(tO[t], a, b, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(tO[t], a, b, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit w = get_unit(u, p);
+        if (w.nb <= 0) continue;
+        ok = mbar_wait(&sm.q_full[0], nunit & 1, g) && mbar_wait(&sm.q_full[1], nunit & 1, g);
+        if (!ok) break;
+        // first K block
+        uint32_t sk = seq % C::NS;
+        ok = mbar_wait(&sm.kv_full[sk], (seq / C::NS) & 1, g);
+        if (!ok) break;
+        tc_fence_after();
+        ++seq;
+        issue_s(0, kv_addr0 + sk * C::TILE_BYTES);
+        tc_commit(&sm.s_full[0]);
+        issue_s(1, kv_addr0 + sk * C::TILE_BYTES);
+        tc_commit(&sm.s_full[1]);
+        tc_commit(&sm.kv_empty[sk]);
+        for (int j = 0; j < w.nb && ok; ++j) {
+          const uint32_t sv = seq % C::NS;
+          ok = mbar_wait(&sm.kv_full[sv], (seq / C::NS) & 1, g);
+          if (!ok) break;
+          ++seq;
+          const bool has_next = j + 1 < w.nb;
+          const uint32_t skn = seq % C::NS;
+          for (int t = 0; t < 2 && ok; ++t) {
+            ok = mbar_wait(&sm.p_full[t], pcnt[t] & 1, g);
+            if (!ok) break;
+            ++pcnt[t];
+            if (j == 0 && nunit > 0) {
+              ok = mbar_wait(&sm.o_empty[t], (nunit - 1) & 1, g);
+              if (!ok) break;
+            }
+            tc_fence_after();
+            issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0);
+            if (!has_next) tc_commit(&sm.o_full[t]);
+            if (has_next) {
+              if (t == 0) {
+                ok = mbar_wait(&sm.kv_full[skn], (seq / C::NS) & 1, g);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              issue_s(t, kv_addr0 + skn * C::TILE_BYTES);
+              tc_commit(&sm.s_full[t]);
+            }
+          }
+          if (!ok) break;
+          tc_commit(&sm.kv_empty[sv]);
+          if (has_next) {
+            tc_commit(&sm.kv_empty[skn]);
+            ++seq;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&sm.q_empty[0]);
+        tc_commit(&sm.q_empty[1]);
+        ++nunit;
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      tc_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, g_drain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;                 // tile of this warpgroup
+    const int r = ((warp & 3) << 5) + lane;  // row within the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+    const uint32_t tS = tmem + (t == 0 ? C::TM_S0 : C::TM_S1) + lane_off;
+    const uint32_t tO = tmem + (t == 0 ? C::TM_O0 : C::TM_O1) + lane_off;
+    const float sl2 = p.scale_log2;
+    uint32_t scnt = 0, nunit = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit w = get_unit(u, p);
+      const int row = w.m0[t] + r;
+      const bool row_valid = row < p.Lq;
+      float m_run = -INFINITY, l_run = 0.f;
+      if (w.nb > 0) {
+        int lo, hi;
+        key_range(row, p, lo, hi);
+        for (int j = 0; j < w.nb; ++j) {
+          ok = mbar_wait(&sm.s_full[t], scnt & 1, g);
+          if (!ok) break;
+          ++scnt;
+          tc_fence_after();
+          float s[kBN];
+#pragma unroll
+          for (int c = 0; c < kBN / 32; ++c) {
+            uint32_t raw[32];
+            tmem_ld32(tS + c * 32, raw);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[i]);
+          }
+          const int key0 = (w.kb_lo + j) * kBN;
+          if (!(lo <= key0 && key0 + kBN <= hi)) {
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) {
+              const int key = key0 + c;
+              if (key < lo || key >= hi) s[c] = -INFINITY;
+            }
+          }
+          float mx = s[0];
+#pragma unroll
+          for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+          const float m_blk = mx * sl2;
+          float alpha = 1.f;
+          if (m_blk > m_run + kRescaleThreshold) {
+            alpha = ex2_approx(m_run - m_blk);  // m_run = -inf -> 0
+            m_run = m_blk;
+          }
+          l_run *= alpha;
+          const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+          float rs = 0.f;
+          if (FP8) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < kBN; c += 4) {
+              const float p0 = ex2_approx(fmaf(s[c + 0], sl2, neg_m));
+              const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg_m));
+              const float p2 = ex2_approx(fmaf(s[c + 2], sl2, neg_m));
+              const float p3 = ex2_approx(fmaf(s[c + 3], sl2, neg_m));
+              const uint16_t lo = pack_e4m3x2(p0, p1), hi = pack_e4m3x2(p2, p3);
+              pk[c / 4] = (uint32_t)lo | ((uint32_t)hi << 16);
+              rs += sum_e4m3x4(lo, hi);  // the row sum sees the same rounded P as the MMA
+            }
+            tmem_st32(tS, pk);
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t pk[32];
+#pragma unroll
+              for (int c = 0; c < 64; c += 2) {
+                const float p0 = ex2_approx(fmaf(s[h * 64 + c], sl2, neg_m));
+                const float p1 = ex2_approx(fmaf(s[h * 64 + c + 1], sl2, neg_m));
+                pk[c / 2] = pack_bf16x2(p0, p1);
+                rs += sum_bf16x2(pk[c / 2]);  // the row sum sees the same rounded P as the MMA
+              }
+              tmem_st32(tS + h * 32, pk);
+            }
+          }
+          l_run += rs;
+          // Rescale the accumulator when the running max moved.  The previous
+          // P.V of this tile has completed: it was issued before this S.
+          const bool need = (j > 0) && (alpha != 1.f);
+          if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t raw[32];
+              tmem_ld32(tO + c * 32, raw);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+              tmem_st32(tO + c * 32, raw);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&sm.p_full[t]);
+        }
+        if (!ok) break;
+        ok = mbar_wait(&sm.o_full[t], nunit & 1, g);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // Epilogue: O = acc / sum (bf16), LSE = (max + log2 sum) * ln 2.
+      const float inv_l = (l_run > 0.f) ? p.out_scale / l_run : 0.f;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)w.bh[t] * p.Lq + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t raw[32];
+        if (w.nb > 0) {
+          tmem_ld32(tO + c * 32, raw);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) raw[i] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(raw[2 * i]) * inv_l, __uint_as_float(raw[2 * i + 1]) * inv_l);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (row_valid && p.lse != nullptr)
+        p.lse[(size_t)w.bh[t] * p.Lq + row] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      if (w.nb > 0) {
+        tc_fence_before();
+        mbar_arrive(&sm.o_empty[t]);
+        ++nunit;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [outer, rows, inner] row-major tensor, box of 128 rows x (128 bytes).
+bool encode_3d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uint64_t rows, uint64_t outer) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  const uint64_t el = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {inner, rows, outer};
+  cuuint64_t strides[2] = {inner * el, inner * rows * el};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / el), (cuuint32_t)kBM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool FP8>
+int run(const PrefillArgs& a, cudaStream_t stream) {
+  using C = Cfg<D, FP8>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -3;
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(prefill_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return -3;
+    attr_set[dev] = true;
+  }
+  Params p{};
+  p.o = a.o;
+  p.lse = a.lse;
+  p.B = a.B;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.Lq = a.Lq;
+  p.Lk = a.Lk;
+  p.group = a.Hq / a.Hkv;
+  p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
+  if (p.pair_heads) {
+    p.n_pairs = a.B * (a.Hq / 2);
+    p.n_mgroups = (a.Lq + kBM - 1) / kBM;
+  } else {
+    p.n_pairs = a.B * a.Hq;
+    p.n_mgroups = (a.Lq + 2 * kBM - 1) / (2 * kBM);
+  }
+  p.n_units = p.n_pairs * p.n_mgroups;
+  p.causal = a.causal;
+  p.window = a.window > 0 ? a.window : 0;
+  const float log2e = 1.4426950408889634f;
+  p.scale_log2 = a.scale * log2e * (FP8 ? a.q_descale * a.k_descale : 1.f);
+  p.out_scale = FP8 ? a.v_descale : 1.f;
+  p.status = device_status_word();
+  if (!p.status) return -3;
+  p.timeout_ns = wait_timeout_ns();
+
+  CUtensorMap tq, tk, tv;
+  const bool have_k = a.Lk > 0;
+  if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq)) return -3;
+  // With no keys nothing is loaded from K/V; describe Q instead of an empty tensor.
+  if (!encode_3d(&tk, have_k ? a.k : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
+    return -3;
+  if (!encode_3d(&tv, have_k ? a.v : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
+    return -3;
+  const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+  prefill_kernel<D, FP8><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+}  // namespace
+
+int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.fp8) {
+    if (a.D == 128) return run<128, true>(a, stream);
+    return -2;
+  }
+  if (a.D == 128) return run<128, false>(a, stream);
+  if (a.D == 64) return run<64, false>(a, stream);
+  return -2;
+}
+
+}  // namespace attn

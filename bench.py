@@ -1,0 +1,450 @@
+"""Benchmark of the attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic inputs:
+  1. fused prefill: GQA causal attention, B=4, Hq=32, Hkv=8, L=4096, D=128, bf16
+     (attn_fwd: tile loads, S = QK^T, masks with block skipping, online softmax,
+     P.V, epilogue);
+  2. paged decode: MQA, B=64 sequences, Hq=32, Hkv=1, D=128, lengths uniform in
+     [512, 8192], 16-token pages behind a permuted block table
+     (attn_decode_paged: split + combine).
+
+The headline ``value`` is prefill TFLOP/s (FLOPs counted as the causal mask
+requires); decode HBM GB/s is reported beside it.  Both come from CUDA events
+recorded around each kernel launch on the launching stream inside the timed
+region.  ``--gpus N`` under torchrun runs N independent replicas (the path has
+no exchange step), times on the device and takes the max over ranks.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import (FP8_CAUSAL, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, decode_inputs,  # noqa: E402
+                       prefill_inputs, prefill_inputs_fp8, seed_of)
+from workloads.accounting import decode_bytes, prefill_bytes, prefill_flops  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (prefill) & decode HBM GB/s, % of B200 roofline"
+PREFILL = GQA_CAUSAL
+DECODE = MQA_DECODE
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' side measurements")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle baseline")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------ distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu):
+        self.gpu = gpu  # nvidia-smi id: "GPU-<uuid>" or an index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"attn_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "", 1).isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        load = [x for x in sm if x > 500] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- CPU baseline
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_oracle_prefill(budget_s: float):
+    """Times the float64 oracle on whole heads of the prefill workload until
+    the budget is spent (at least one head).  Returns (TFLOP/s, heads, seconds)."""
+    import oracle
+    q, k, v = prefill_inputs(PREFILL, seed_of(1))
+    per_head = prefill_flops(PREFILL) / (PREFILL.B * PREFILL.Hq)
+    heads = 0
+    t0 = time.perf_counter()
+    while True:
+        b, h = divmod(heads, PREFILL.Hq)
+        oracle.attention(q, k, v, PREFILL.scale, PREFILL.causal, PREFILL.window, heads=[h], batches=[b])
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or heads >= PREFILL.B * PREFILL.Hq:
+            break
+    return per_head * heads / el / 1e12, heads, el
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    import attention_flash_attn_02_b200 as attn
+    attn.load()
+    dev = torch.device("cuda", local)
+    peaks, peak_src = measured_peaks()
+
+    # inputs resident in HBM before the timed region
+    qh, kh, vh = prefill_inputs(PREFILL, seed_of(1))
+    q, k, v = qh.to(dev), kh.to(dev), vh.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    kv = decode_inputs(DECODE, seed_of(2))
+    dq, dkp, dvp = kv.q.to(dev), kv.k_pages.to(dev), kv.v_pages.to(dev)
+    dbt, dsl = kv.block_table.to(dev), kv.seq_lens.to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty(dq.shape[:2], dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.attn_decode_workspace_bytes(DECODE.B, DECODE.Hq, kv.max_pages, DECODE.D),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        attn.attn_fwd(q, k, v, PREFILL.scale, PREFILL.causal, PREFILL.window, o=o, lse=lse)
+        if ev is not None:
+            ev[1].record(stream)
+        flush.zero_()  # evict L2 so decode reads its cache from HBM
+        if ev is not None:
+            ev[2].record(stream)
+        attn.attn_decode_paged(dq, dkp, dvp, dbt, dsl, DECODE.scale, o=do, lse=dlse, workspace=ws)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = attn.attn_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"kernel status {attn.attn_status_str(st)} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    st = attn.attn_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"kernel status {attn.attn_status_str(st)} during the timed region")
+
+    region_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    pre_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world, dev)
+    dec_ms = max_over_ranks(sum(e[2].elapsed_time(e[3]) for e in evs), world, dev)
+    K = args.steps
+    pf = prefill_flops(PREFILL)
+    db = decode_bytes(DECODE, kv.seq_lens.tolist())
+    value = world * pf * K / (pre_ms / 1e3) / 1e12            # TFLOP/s, all ranks
+    dec_gbs = world * db * K / (dec_ms / 1e3) / 1e9
+    per_launch_pre_ms = pre_ms / K
+    achieved_pre = pf / (per_launch_pre_ms / 1e3) / 1e12        # per GPU, per launch
+    achieved_dec = db / (dec_ms / K / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    hq, hk, hv = pin(qh), pin(kh), pin(vh)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    hdq, hdk, hdv = pin(kv.q), pin(kv.k_pages), pin(kv.v_pages)
+    hbt, hsl = pin(kv.block_table), pin(kv.seq_lens)
+    hdo = torch.empty(do.shape, dtype=do.dtype).pin_memory()
+    hdl = torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv, hbt, hsl))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdo, hdl))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        attn.attn_fwd(q, k, v, PREFILL.scale, PREFILL.causal, PREFILL.window, o=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        dq.copy_(hdq, non_blocking=True)
+        dkp.copy_(hdk, non_blocking=True)
+        dvp.copy_(hdv, non_blocking=True)
+        dbt.copy_(hbt, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        attn.attn_decode_paged(dq, dkp, dvp, dbt, dsl, DECODE.scale, o=do, lse=dlse, workspace=ws)
+        hdo.copy_(do, non_blocking=True)
+        hdl.copy_(dlse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = world * pf * K / (e2e_ms / 1e3) / 1e12
+
+    # ---- side measurements of the other workloads (not part of the step)
+    extra = {}
+    if not args.no_extra:
+        extra = side_workloads(attn, dev, peaks, world)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, heads, secs = cpu_oracle_prefill(args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 oracle, {heads} whole (batch, head) pairs of the prefill workload "
+                         f"(4096 causal rows each), {secs:.1f} s on the host"}
+
+    peak_t = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(region_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) q/k/v cast to bf16; decode lengths U[512,8192], permuted page table",
+        "config": {
+            "workload": "prefill gqa_causal B4 Hq32 Hkv8 L4096 D128 + paged decode mqa B64 Hq32 Hkv1 D128 len[512,8192] page16",
+            "prefill": PREFILL.name, "decode": DECODE.name,
+            "l2": "prefill inputs 201 MB > L2; 256 MB buffer written before each decode",
+            "parallelism": f"replicas{world}",
+        },
+        "roofline": {
+            "bound": "tensor", "kernel": "prefill_kernel<128,bf16>",
+            "achieved": round(achieved_pre, 2), "peak": peak_t, "unit": "TFLOP/s",
+            "frac": round(achieved_pre / peak_t, 4),
+            "frac_of_sustained": round(achieved_pre / peaks["bf16_tflops_sustained"], 4),
+            "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "traffic": None,
+        },
+        "decode": {
+            "value": round(dec_gbs, 1), "unit": "GB/s", "workload": DECODE.name,
+            "us_per_call": round(dec_ms / K * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved_dec, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(achieved_dec / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peak_src} hbm_gbs", "traffic": None},
+        },
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+        "workloads": extra,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def side_workloads(attn, dev, peaks, world):
+    """Per-launch TFLOP/s of the sliding-window and FP8 workloads (median of
+    5 launches after 2 warm-ups; inputs larger than L2)."""
+    import torch
+    out = {}
+    for shape, idx in ((SWA_CAUSAL, 3), (FP8_CAUSAL, 4)):
+        if shape.fp8:
+            q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, seed_of(idx))
+            q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+            fn = lambda: attn.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, shape.scale, shape.causal, shape.window)  # noqa
+        else:
+            q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(idx))]
+            fn = lambda: attn.attn_fwd(q, k, v, shape.scale, shape.causal, shape.window)  # noqa
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = max_over_ranks(statistics.median(ts), world, dev)
+        tf = prefill_flops(shape) / (ms / 1e3) / 1e12
+        entry = {"TFLOP/s": round(tf, 1), "ms": round(ms, 3), "bytes_MB": round(prefill_bytes(shape) / 1e6, 1)}
+        if shape.fp8:
+            entry["frac_of_bf16_peak"] = round(tf / peaks["bf16_tflops"], 4)
+            entry["note"] = "no measured FP8 peak; nominal dense FP8 is 2x bf16"
+        else:
+            entry["frac"] = round(tf / peaks["bf16_tflops"], 4)
+        out[shape.name] = entry
+        del fn
+        torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------- reference
+def run_reference(args):
+    """The float64 oracle on the host cores, each step a bounded sample of
+    the same workload: one whole (batch, head) of the prefill and one
+    sequence of the decode."""
+    rank, world, _ = dist_env()
+    if world > 1 and rank != 0:
+        return
+    import oracle
+    q, k, v = prefill_inputs(PREFILL, seed_of(1))
+    kv = decode_inputs(DECODE, seed_of(2))
+    per_head = prefill_flops(PREFILL) / (PREFILL.B * PREFILL.Hq)
+
+    def step(i):
+        b, h = divmod(i % (PREFILL.B * PREFILL.Hq), PREFILL.Hq)
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, PREFILL.scale, PREFILL.causal, PREFILL.window, heads=[h], batches=[b])
+        t1 = time.perf_counter()
+        sb = i % DECODE.B
+        oracle.paged_decode(kv.q[sb:sb + 1], kv.k_pages, kv.v_pages, kv.block_table[sb:sb + 1],
+                            kv.seq_lens[sb:sb + 1], DECODE.scale)
+        return t1 - t0, time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        step(i)
+    pre = tot = 0.0
+    for i in range(args.steps):
+        a, b = step(args.warmup + i)
+        pre += a
+        tot += b
+    value = per_head * args.steps / pre / 1e12
+    line = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 5), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
+        "config": {"workload": "prefill gqa_causal B4 Hq32 Hkv8 L4096 D128 + paged decode mqa B64 Hq32 Hkv1 D128",
+                   "prefill": PREFILL.name, "decode": DECODE.name, "parallelism": "host"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": "each step: one whole (batch, head) of the prefill workload and one decode "
+                                   "sequence, float64 oracle"},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

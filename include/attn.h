@@ -1,0 +1,188 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) fused attention library
+ * (libattn_sm100.so).
+ *
+ * Two operations, both forward only, both on one GPU:
+ *
+ *   attn_fwd / attn_fwd_fp8   fused, tiled scaled-dot-product attention
+ *                             O = softmax(scale * Q K^T + mask) V, with the
+ *                             per-row log-sum-exp, computed with the online
+ *                             softmax recurrence (running row max and sum,
+ *                             accumulator rescaled at each K/V block) so the
+ *                             score matrix never reaches HBM.
+ *   attn_decode_paged         one query token per sequence against a KV cache
+ *                             held in fixed-size pages addressed through a
+ *                             block table, split over the cache and merged by
+ *                             log-sum-exp.
+ *
+ * Sources (page title, section):
+ *   - "003-注意力机制详解：从基础Attention到DeepSeek的优化策略" (lakecityint.com),
+ *     §一 attention_naive / safe_softmax (the definition), §二 the tiled
+ *     FlashAttention loop (online softmax), §三.1 mixed precision (fp16/bf16
+ *     operands, fp32 softmax and accumulation), §三.2 sliding window.
+ *   - "LLM 中的 Attention 实现及优化" (zeeklog.com): MQA/GQA with repeat_kv and
+ *     the (batch, heads, seqlen, head_dim) layout; the KV-cache size formula;
+ *     sliding-window attention; PagedAttention.
+ *   - MQA / GQA / Flash Attention article (tqpw.cn) §2.1 (MQA), §3.1 (GQA,
+ *     h % g == 0), §4.1-4.2 (tiling into SRAM, online softmax, one fused
+ *     kernel).
+ *   - "注意力机制深度优化" (kler.cn) §一.1 (FP8 e4m3), §一.2 (skipping the
+ *     upper-right causal triangle).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers unless stated otherwise.  The caller owns
+ *     every buffer (inputs, outputs and the decode workspace); the library
+ *     allocates no device memory on any call.  Its only device state is one
+ *     status word per GPU, created when the library is loaded.
+ *   - All launches are asynchronous on the caller's CUDA stream `stream`
+ *     (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - A call returns ATTN_OK once its kernels are enqueued.  Argument errors
+ *     are detected on the host before anything is launched and return
+ *     ATTN_ERR_INVALID / ATTN_ERR_UNSUPPORTED with nothing written.  A CUDA
+ *     launch failure returns ATTN_ERR_CUDA.  Errors found by the kernels
+ *     themselves (a bounded wait that ran out, an out-of-range page id in
+ *     bounds-check mode) are recorded in the device status word and reported
+ *     by attn_last_device_error().  The kernels never trap.
+ *   - Tensors are contiguous, row-major, with a 16-byte aligned base.
+ */
+#ifndef ATTN_SM100_H
+#define ATTN_SM100_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+#define ATTN_API extern "C" __attribute__((visibility("default")))
+#else
+#define ATTN_API __attribute__((visibility("default")))
+#endif
+
+typedef void* attn_stream_t; /* cudaStream_t of the caller */
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = -1,     /* bad argument (shape, pointer, alignment) */
+  ATTN_ERR_UNSUPPORTED = -2, /* valid but not built (e.g. head_dim 96)   */
+  ATTN_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed         */
+  ATTN_ERR_TIMEOUT = -4,     /* a kernel's bounded wait ran out           */
+  ATTN_ERR_BOUNDS = -5       /* bounds-check mode found a bad index       */
+};
+
+/*
+ * attn_fwd -- bf16 fused attention forward (prefill).
+ *
+ *   q    [B, Hq,  Lq, D] bf16     k, v [B, Hkv, Lk, D] bf16
+ *   o    [B, Hq,  Lq, D] bf16 (written)
+ *   lse  [B, Hq,  Lq]    fp32 (written; may be NULL): natural-log
+ *        log-sum-exp of the scaled, masked logits of each row.
+ *
+ * Layout (batch, heads, seqlen, head_dim) as produced by
+ * view(...).transpose(1, 2) in the zeeklog page's GQA code.  Query head h reads
+ * K/V head h / (Hq / Hkv): MHA (Hkv == Hq), GQA (Hq % Hkv == 0) and MQA
+ * (Hkv == 1).  Scores are scale * q.k accumulated in fp32; softmax in fp32; P
+ * is rounded to bf16 for the P.V product; O is accumulated in fp32 and rounded
+ * to bf16 once (mixed-precision scheme of the lakecityint.com page §三.1).
+ *
+ * Masks:
+ *   causal = 0: every query sees all Lk keys.
+ *   causal = 1: query i sees keys 0 .. i + (Lk - Lq) (the triangle is aligned
+ *     to the bottom-right corner; with Lq == Lk this is keys 0..i).  K/V blocks
+ *     entirely above the diagonal are never loaded or multiplied.
+ *   window W > 0 (requires causal = 1): query i sees the W keys
+ *     max(0, i' - W + 1) .. i' with i' = i + (Lk - Lq).  Blocks entirely before
+ *     the window are never loaded.  window <= 0: no window.
+ * A row that sees no key (only possible when Lq > Lk with causal = 1, or
+ * Lk == 0) gets O = 0 and LSE = -inf.
+ *
+ * Supported: D in {64, 128}; 1 <= Hkv <= Hq, Hq % Hkv == 0; B, Lq >= 0;
+ * Lk >= 0; any Lq, Lk (ragged tails are handled).  Returns ATTN_ERR_INVALID
+ * for bad shapes, NULL or misaligned pointers, window > 0 without causal;
+ * ATTN_ERR_UNSUPPORTED for other D.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                      float scale, int causal, int window, attn_stream_t stream);
+
+/*
+ * attn_fwd_fp8 -- the same operation on float8_e4m3fn inputs (the e4m3 FP8
+ * format of the kler.cn page §一.1), bf16 output.
+ *
+ *   q, k, v  e4m3 bytes, same shapes/layout as attn_fwd; o bf16; lse fp32.
+ *   q_descale, k_descale, v_descale: per-tensor scales, i.e. the real value of
+ *   an element is e4m3_value * descale.  The logits are
+ *   scale * q_descale * k_descale * (q8 . k8); P is quantised to e4m3 for the
+ *   P.V product (values in [0, 256]); O is multiplied by v_descale.
+ *
+ * Supported: D == 128 only (ATTN_ERR_UNSUPPORTED otherwise).
+ */
+ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                          float scale, int causal, int window,
+                          float q_descale, float k_descale, float v_descale,
+                          attn_stream_t stream);
+
+/*
+ * attn_decode_workspace_bytes -- size of the scratch buffer attn_decode_paged
+ * needs for these sizes (split partials: per sequence, per split of 512
+ * cached tokens, per query head, D + 1 floats).  Host only; never fails (0 for empty shapes).
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D);
+
+/*
+ * attn_decode_paged -- single-token decode against a paged KV cache
+ * (PagedAttention section of the zeeklog page: non-contiguous small-block KV
+ * storage), split over the cache and merged by log-sum-exp.
+ *
+ *   q           [B, Hq, D] bf16, one query token per sequence
+ *   k_pages     [num_pages, page_size, Hkv, D] bf16, shared pool
+ *   v_pages     [num_pages, page_size, Hkv, D] bf16
+ *   block_table [B, max_pages_per_seq] int32: page id of each page of each
+ *               sequence (entries past a sequence's length are not read)
+ *   seq_lens    [B] int32 (device), 0 <= seq_lens[b] <= max_pages_per_seq *
+ *               page_size (longer lengths are clamped to that)
+ *   o           [B, Hq, D] bf16 (written)
+ *   lse         [B, Hq] fp32 (written; may be NULL)
+ *   workspace   caller-owned device scratch of at least
+ *               attn_decode_workspace_bytes(B, Hq, max_pages_per_seq, D) bytes;
+ *               its contents on entry do not matter.
+ *
+ * The single query sees every cached key (causal alignment at the
+ * bottom-right corner).  seq_lens[b] == 0 gives O = 0 and LSE = -inf.
+ * Supported: page_size == 16, D == 128, Hq % Hkv == 0 and Hq / Hkv <= 32.
+ * Page ids are trusted unless bounds-check mode is on (attn_set_debug), in
+ * which case an id outside [0, num_pages) is skipped and reported as
+ * ATTN_ERR_BOUNDS by attn_last_device_error().
+ */
+ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                               const int* block_table, const int* seq_lens, void* o, float* lse,
+                               int B, int Hq, int Hkv, int D, int page_size, int num_pages,
+                               int max_pages_per_seq, float scale,
+                               void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_last_device_error -- synchronises `stream`, then returns and clears the
+ * status word the kernels write on the current device: ATTN_OK,
+ * ATTN_ERR_TIMEOUT (a bounded wait inside a kernel ran out; the kernel
+ * released its resources and returned), ATTN_ERR_BOUNDS, or ATTN_ERR_CUDA if
+ * the synchronisation itself failed.
+ */
+ATTN_API int attn_last_device_error(attn_stream_t stream);
+
+/* attn_status_str -- static, human-readable name of a status code. */
+ATTN_API const char* attn_status_str(int status);
+
+/*
+ * attn_set_debug -- process-wide debug switches for later launches.
+ *   flags bit 0 (ATTN_DEBUG_BOUNDS): decode checks every page id against
+ *                num_pages and every token against seq_len.
+ *   wait_timeout_ns: limit of every bounded wait inside the kernels
+ *                (0 = the default of 2 s).
+ * Returns the previous flags.
+ */
+#define ATTN_DEBUG_BOUNDS 1
+ATTN_API int attn_set_debug(int flags, unsigned long long wait_timeout_ns);
+
+/* attn_version -- ABI version of this header (currently 1). */
+ATTN_API int attn_version(void);
+
+#endif /* ATTN_SM100_H */

@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA kernels (through the C ABI) against the float64 oracle
+on the same seeded inputs.
+
+Tolerances (bf16 output): max |O - O_ref| <= 1e-2, mean <= 1e-3, and
+|LSE - LSE_ref| <= 1e-3; FP8 inputs: 5e-2 / 5e-3 on O, 1e-3 on LSE.  The
+bf16 rounding of O alone contributes up to half an ulp (3.9e-3 for |O| in
+[1, 2)); the rest comes from fp32 accumulation and the bf16 (or e4m3)
+rounding of P before the P.V product.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import (FP8_CAUSAL, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, TINY_MHA, DecodeShape,
+                       PrefillShape, decode_inputs, prefill_inputs, prefill_inputs_fp8, seed_of)
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = (1e-2, 1e-3)
+FP8_TOL = (5e-2, 5e-3)
+LSE_TOL = 1e-3
+
+
+def _errs(o_gpu, o_ref, lse_gpu, lse_ref):
+    o_gpu = o_gpu.double().cpu().numpy()
+    lse_gpu = lse_gpu.double().cpu().numpy()
+    d = np.abs(o_gpu - o_ref)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse_gpu), fin), "LSE finiteness differs (empty rows)"
+    dl = np.abs(lse_gpu[fin] - lse_ref[fin]) if fin.any() else np.zeros(1)
+    return float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0, float(dl.max())
+
+
+def _check(o_gpu, o_ref, lse_gpu, lse_ref, tol=BF16_TOL, what=""):
+    mx, mean, dl = _errs(o_gpu, o_ref, lse_gpu, lse_ref)
+    assert mx <= tol[0] and mean <= tol[1] and dl <= LSE_TOL, \
+        f"{what}: max {mx:.3e} mean {mean:.3e} lse {dl:.3e}"
+    # rows with no visible key must be exactly zero
+    empty = ~np.isfinite(lse_ref)
+    if empty.any():
+        assert np.all(o_gpu.float().cpu().numpy()[empty] == 0)
+    return mx, mean, dl
+
+
+def _run_prefill(lib, shape: PrefillShape, seed: int):
+    q, k, v = prefill_inputs(shape, seed)
+    o, lse = lib.attn_fwd(q.cuda(), k.cuda(), v.cuda(), shape.scale, shape.causal, shape.window)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    return q, k, v, o, lse
+
+
+def test_tiny_mha_exact_definition(lib):
+    shape = TINY_MHA
+    q, k, v, o, lse = _run_prefill(lib, shape, seed_of(0))
+    o_ref, l_ref = oracle.attention(q, k, v, shape.scale, shape.causal, shape.window)
+    _check(o, o_ref, lse, l_ref, what=shape.name)
+
+
+SWEEP = []
+for D in (64, 128):
+    for (Hq, Hkv) in ((2, 2), (4, 1), (8, 2), (3, 1)):
+        for L in (1, 17, 127, 128, 129, 300):
+            for causal in (False, True):
+                SWEEP.append((1, Hq, Hkv, L, L, D, causal, 0))
+SWEEP += [
+    (3, 4, 4, 1000, 1000, 128, True, 0),
+    (1, 8, 1, 257, 257, 128, False, 0),
+    (2, 32, 1, 200, 200, 128, True, 0),     # MQA, group 32
+    (1, 4, 2, 100, 300, 128, True, 0),      # Lq < Lk, bottom-right causal
+    (1, 4, 2, 100, 300, 64, False, 0),
+    (1, 4, 2, 300, 100, 128, True, 0),      # Lq > Lk: first rows see no key
+    (1, 2, 2, 50, 0, 128, False, 0),        # no keys at all
+]
+for W in (1, 2, 127, 128, 129, 300, 5000):
+    SWEEP.append((1, 4, 2, 600, 600, 128, True, W))
+    SWEEP.append((1, 3, 3, 300, 300, 64, True, W))
+SWEEP.append((2, 8, 2, 1000, 1300, 128, True, 200))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,window", SWEEP)
+def test_prefill_sweep(lib, B, Hq, Hkv, Lq, Lk, D, causal, window):
+    shape = PrefillShape("sweep", B, Hq, Hkv, Lq, Lk, D, causal, window)
+    q, k, v, o, lse = _run_prefill(lib, shape, 7 + Lq + 3 * Lk + D + window)
+    o_ref, l_ref = oracle.attention(q, k, v, shape.scale, causal, window)
+    _check(o, o_ref, lse, l_ref, what=str(shape))
+
+
+def test_window_at_least_length_equals_causal_on_gpu(lib):
+    shape = PrefillShape("w", 1, 4, 2, 333, 333, 128, True, 0)
+    q, k, v = prefill_inputs(shape, 5)
+    a = lib.attn_fwd(q.cuda(), k.cuda(), v.cuda(), shape.scale, True, 0)
+    b = lib.attn_fwd(q.cuda(), k.cuda(), v.cuda(), shape.scale, True, 333)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_causal_row_zero_and_window_one_are_exact(lib):
+    """Row 0 under a causal mask (and every row with W = 1) sees one key, so
+    O equals that bf16 V row exactly."""
+    shape = PrefillShape("w1", 1, 4, 2, 256, 256, 128, True, 1)
+    q, k, v = prefill_inputs(shape, 6)
+    o, lse = lib.attn_fwd(q.cuda(), k.cuda(), v.cuda(), shape.scale, True, 1)
+    torch.cuda.synchronize()
+    vr = v.repeat_interleave(2, dim=1)
+    assert torch.equal(o.cpu(), vr)
+    o2, _ = lib.attn_fwd(q.cuda(), k.cuda(), v.cuda(), shape.scale, True, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(o2[:, :, 0].cpu(), vr[:, :, 0])
+
+
+def _sampled_rows(L, n, seed):
+    g = np.random.default_rng(seed)
+    rows = set(g.choice(L, size=n, replace=False).tolist())
+    rows |= {0, 1, 127, 128, L - 1}
+    return sorted(r for r in rows if r < L)
+
+
+@pytest.mark.parametrize("idx,shape", [(1, GQA_CAUSAL), (3, SWA_CAUSAL)])
+def test_full_size_prefill_sampled_rows(lib, idx, shape):
+    """Full workload on the GPU; the oracle computes sampled rows of a few
+    (batch, head) pairs, one by one."""
+    q, k, v, o, lse = _run_prefill(lib, shape, seed_of(idx))
+    rows = _sampled_rows(shape.Lq, 24, idx)
+    for b, heads in ((0, [0, 1, 5]), (shape.B - 1, [shape.Hq - 1, shape.Hq - 4])):
+        o_ref, l_ref = oracle.attention(q, k, v, shape.scale, shape.causal, shape.window,
+                                        rows=rows, heads=heads, batches=[b])
+        _check(o[b][heads][:, rows], o_ref[0], lse[b][heads][:, rows], l_ref[0], what=shape.name)
+
+
+def test_fp8_small(lib):
+    shape = PrefillShape("fp8_small", 1, 4, 4, 700, 700, 128, True, fp8=True)
+    q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, 11)
+    o, lse = lib.attn_fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), sq, sk, sv, shape.scale, True, 0)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    o_ref, l_ref = oracle.attention_fp8(q8, k8, v8, sq, sk, sv, shape.scale, True)
+    _check(o, o_ref, lse, l_ref, FP8_TOL, what="fp8 small")
+
+
+def test_fp8_full_size_sampled_rows(lib):
+    shape = FP8_CAUSAL
+    q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, seed_of(4))
+    o, lse = lib.attn_fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), sq, sk, sv, shape.scale, True, 0)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    rows = _sampled_rows(shape.Lq, 16, 4)
+    heads = [0, 13, 31]
+    o_ref, l_ref = oracle.attention_fp8(q8, k8, v8, sq, sk, sv, shape.scale, True,
+                                        rows=rows, heads=heads, batches=[0])
+    _check(o[0][heads][:, rows], o_ref[0], lse[0][heads][:, rows], l_ref[0], FP8_TOL, what=shape.name)
+
+
+# ------------------------------------------------------------------ decode
+def _run_decode(lib, kv, scale):
+    d = {n: getattr(kv, n).cuda() for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+    o, lse = lib.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], scale)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    return o, lse
+
+
+def test_decode_full_workload(lib):
+    shape = MQA_DECODE
+    kv = decode_inputs(shape, seed_of(2))
+    o, lse = _run_decode(lib, kv, shape.scale)
+    o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, o_ref, lse, l_ref, what=shape.name)
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv", [
+    ([1, 15, 16, 17, 512, 513, 8192, 0], 32, 1),
+    ([3, 100, 1000, 2049], 32, 4),
+    ([700, 1, 64], 16, 2),
+    ([5000, 31], 8, 8),
+    ([0, 0], 32, 1),
+])
+def test_decode_edge_lengths(lib, lens, Hq, Hkv):
+    shape = DecodeShape("edge", B=len(lens), Hq=Hq, Hkv=Hkv, D=128, len_lo=1, len_hi=1)
+    kv = decode_inputs(shape, 99 + sum(lens), seq_lens=lens, extra_pages=5)
+    o, lse = _run_decode(lib, kv, shape.scale)
+    o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, o_ref, lse, l_ref, what=str(lens))
+
+
+def test_decode_invariant_to_page_permutation(lib):
+    shape = DecodeShape("perm", B=4, Hq=32, Hkv=1, D=128, len_lo=100, len_hi=900)
+    kv = decode_inputs(shape, 5)
+    o1, l1 = _run_decode(lib, kv, shape.scale)
+    perm = torch.randperm(kv.num_pages, generator=torch.Generator().manual_seed(1))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(kv.num_pages)
+    kp = torch.empty_like(kv.k_pages)
+    vp = torch.empty_like(kv.v_pages)
+    kp[inv] = kv.k_pages
+    vp[inv] = kv.v_pages
+    kv.k_pages, kv.v_pages = kp, vp
+    kv.block_table = inv[kv.block_table.long()].int()
+    o2, l2 = _run_decode(lib, kv, shape.scale)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_decode_bounds_check_reports_bad_page(lib):
+    shape = DecodeShape("bounds", B=2, Hq=32, Hkv=1, D=128, len_lo=1, len_hi=1)
+    kv = decode_inputs(shape, 3, seq_lens=[40, 20])
+    kv.block_table[1, 0] = kv.num_pages + 7       # out of the pool
+    prev = lib.attn_set_debug(lib.ATTN_DEBUG_BOUNDS, 0)
+    try:
+        d = {n: getattr(kv, n).cuda() for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+        lib.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], shape.scale)
+        assert lib.attn_last_device_error() == lib.ATTN_ERR_BOUNDS
+        assert lib.attn_last_device_error() == 0      # cleared by the read
+    finally:
+        lib.attn_set_debug(prev, 0)
