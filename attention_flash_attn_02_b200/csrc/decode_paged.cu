@@ -168,7 +168,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
 #pragma unroll
   for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY};
-  float l_part[2] = {0.f, 0.f};  // per-lane partial row sums
+  // per-lane partial row sums: exact fp32 (for the LSE) and of the rounded P
+  // the tensor cores multiply (normalises o)
+  float l_part[2] = {0.f, 0.f}, r_part[2] = {0.f, 0.f};
   const float sl2 = p.scale_log2;
 
   for (int ch = 0; ch < nchunks; ++ch) {
@@ -215,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
         m_run[h] = mx;
       }
       l_part[h] *= alpha[h];
+      r_part[h] *= alpha[h];
     }
     if (alpha[0] != 1.f || alpha[1] != 1.f) {
 #pragma unroll
@@ -236,14 +239,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
         pv[n][1] = ex2_approx(s[n][1] + nm0);
         pv[n][2] = ex2_approx(s[n][2] + nm1);
         pv[n][3] = ex2_approx(s[n][3] + nm1);
+        l_part[0] += pv[n][0] + pv[n][1];
+        l_part[1] += pv[n][2] + pv[n][3];
       }
       pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
       pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
       pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
       pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
       // row sums of the same rounded P the tensor cores multiply
-      l_part[0] += sum_bf16x2(pa[0]) + sum_bf16x2(pa[2]);
-      l_part[1] += sum_bf16x2(pa[1]) + sum_bf16x2(pa[3]);
+      r_part[0] += sum_bf16x2(pa[0]) + sum_bf16x2(pa[2]);
+      r_part[1] += sum_bf16x2(pa[1]) + sum_bf16x2(pa[3]);
     }
     // O += P V over 16 tokens x 128 features
 #pragma unroll
@@ -259,17 +264,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
 
   // Merge the 4 token slices of each query tile through shared memory.
   float* s_o = reinterpret_cast<float*>(smem + kQBytes);        // [8 warps][16 rows][128]
-  float* s_ml = s_o + 8 * 16 * kD;                              // [8 warps][16 rows][2]
+  float* s_ml = s_o + 8 * 16 * kD;                              // [8 warps][16 rows][3]
   {
     const int r0 = lane >> 2;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float l = l_part[h];
+      float l = l_part[h], lr = r_part[h];
       l += __shfl_xor_sync(0xffffffffu, l, 1);
       l += __shfl_xor_sync(0xffffffffu, l, 2);
+      lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+      lr += __shfl_xor_sync(0xffffffffu, lr, 2);
       if ((lane & 3) == 0) {
-        s_ml[(warp * 16 + r0 + 8 * h) * 2 + 0] = m_run[h];
-        s_ml[(warp * 16 + r0 + 8 * h) * 2 + 1] = l;
+        s_ml[(warp * 16 + r0 + 8 * h) * 3 + 0] = m_run[h];
+        s_ml[(warp * 16 + r0 + 8 * h) * 3 + 1] = l;
+        s_ml[(warp * 16 + r0 + 8 * h) * 3 + 2] = lr;
       }
     }
 #pragma unroll
@@ -288,15 +296,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
       const int mtile = row >> 4, r = row & 15;
       float M = -INFINITY;
 #pragma unroll
-      for (int sb = 0; sb < 4; ++sb) M = fmaxf(M, s_ml[((sb * 2 + mtile) * 16 + r) * 2]);
-      float w[4], L = 0.f;
+      for (int sb = 0; sb < 4; ++sb) M = fmaxf(M, s_ml[((sb * 2 + mtile) * 16 + r) * 3]);
+      float w[4], L = 0.f, LR = 0.f;
 #pragma unroll
       for (int sb = 0; sb < 4; ++sb) {
-        const float m = s_ml[((sb * 2 + mtile) * 16 + r) * 2];
+        const float m = s_ml[((sb * 2 + mtile) * 16 + r) * 3];
         w[sb] = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-        L += w[sb] * s_ml[((sb * 2 + mtile) * 16 + r) * 2 + 1];
+        L += w[sb] * s_ml[((sb * 2 + mtile) * 16 + r) * 3 + 1];
+        LR += w[sb] * s_ml[((sb * 2 + mtile) * 16 + r) * 3 + 2];
       }
-      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float inv = LR > 0.f ? 1.f / LR : 0.f;
       const int h = kvh * p.group + row;
       const size_t rec = ((size_t)b * p.Hq + h) * p.max_splits + split;
       float* dst = p.ws_o + rec * kD;

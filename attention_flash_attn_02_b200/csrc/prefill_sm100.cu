@@ -359,7 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit w = get_unit(u, p);
       const int row = w.m0[t] + r;
       const bool row_valid = row < p.Lq;
-      float m_run = -INFINITY, l_run = 0.f;
+      // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
+      // the MMA multiplies (normalises O so its weights sum to one).
+      float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
       if (w.nb > 0) {
         int lo, hi;
         key_range(row, p, lo, hi);
@@ -394,8 +396,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_run = m_blk;
           }
           l_run *= alpha;
+          l_rnd *= alpha;
           const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-          float rs = 0.f;
+          float rs = 0.f, rr = 0.f;
           if (FP8) {
             uint32_t pk[32];
 #pragma unroll
@@ -406,7 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float p3 = ex2_approx(fmaf(s[c + 3], sl2, neg_m));
               const uint16_t lo = pack_e4m3x2(p0, p1), hi = pack_e4m3x2(p2, p3);
               pk[c / 4] = (uint32_t)lo | ((uint32_t)hi << 16);
-              rs += sum_e4m3x4(lo, hi);  // the row sum sees the same rounded P as the MMA
+              rs += (p0 + p1) + (p2 + p3);
+              rr += sum_e4m3x4(lo, hi);
             }
             tmem_st32(tS, pk);
           } else {
@@ -418,12 +422,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float p0 = ex2_approx(fmaf(s[h * 64 + c], sl2, neg_m));
                 const float p1 = ex2_approx(fmaf(s[h * 64 + c + 1], sl2, neg_m));
                 pk[c / 2] = pack_bf16x2(p0, p1);
-                rs += sum_bf16x2(pk[c / 2]);  // the row sum sees the same rounded P as the MMA
+                rs += p0 + p1;
+                rr += sum_bf16x2(pk[c / 2]);
               }
               tmem_st32(tS + h * 32, pk);
             }
           }
           l_run += rs;
+          l_rnd += rr;
           // Rescale the accumulator when the running max moved.  The previous
           // P.V of this tile has completed: it was issued before this S.
           const bool need = (j > 0) && (alpha != 1.f);
@@ -447,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       // Epilogue: O = acc / sum (bf16), LSE = (max + log2 sum) * ln 2.
-      const float inv_l = (l_run > 0.f) ? p.out_scale / l_run : 0.f;
+      const float inv_l = (l_rnd > 0.f) ? p.out_scale / l_rnd : 0.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)w.bh[t] * p.Lq + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

@@ -99,12 +99,12 @@ def measured_peaks():
 class ClockSampler:
     """Samples SM clocks and throttle reasons with nvidia-smi every 200 ms."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu):
-        self.gpu = gpu  # nvidia-smi id: "GPU-<uuid>" or an index
+    def __init__(self, uuid):
+        self.uuid = (uuid or "").lower()  # CUDA uuid of the device under test
         self.proc = None
         self.path = os.path.join("/tmp", f"attn_bench_clocks_{os.getpid()}.csv")
 
@@ -112,7 +112,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -131,6 +131,9 @@ class ClockSampler:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 9:
                 rows.append(parts)
+        uuids = {r[0].lower() for r in rows}
+        mine = [r for r in rows if self.uuid and self.uuid in r[0].lower()]
+        rows = mine if mine else (rows if len(uuids) == 1 else [])
         os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
@@ -222,10 +225,10 @@ def run_ours(args):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+        gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
-        gpu_id = str(local)
-    clocks = ClockSampler(gpu_id)
+        gpu_uuid = ""
+    clocks = ClockSampler(gpu_uuid)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
