@@ -38,7 +38,10 @@ _lib = None
 class AttnError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what} failed: {attn_status_str(status)} ({status})")
+        detail = ""
+        if status == ATTN_ERR_CUDA:
+            detail = " -- " + attn_last_error_message()
+        super().__init__(f"{what} failed: {attn_status_str(status)} ({status}){detail}")
 
 
 def load(path: Optional[str] = None) -> ctypes.CDLL:
@@ -66,6 +69,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_status_str.restype = ctypes.c_char_p
     lib.attn_set_debug.argtypes = [c_int, ctypes.c_ulonglong]
     lib.attn_set_debug.restype = c_int
+    lib.attn_last_error_message.argtypes = []
+    lib.attn_last_error_message.restype = ctypes.c_char_p
     lib.attn_version.argtypes = []
     lib.attn_version.restype = c_int
     _lib = lib
@@ -179,6 +184,10 @@ def attn_last_device_error(stream=None) -> int:
 
 def attn_set_debug(flags: int, wait_timeout_ns: int = 0) -> int:
     return int(load().attn_set_debug(int(flags), int(wait_timeout_ns)))
+
+
+def attn_last_error_message() -> str:
+    return load().attn_last_error_message().decode()
 
 
 def attn_version() -> int:

@@ -7,6 +7,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -49,22 +50,65 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and up_to_date():
+# The prefill kernel redistributes registers between its warpgroups with
+# setmaxnreg; the split assumes this launch register count (see
+# csrc/prefill_sm100.cu).  A different count could make the increase wait
+# forever, so the build refuses to produce such a library.
+PREFILL_LAUNCH_REGS = 168
+
+
+def check_register_counts(ptxas_log: str) -> None:
+    entry = None
+    seen = 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and "prefill_kernel" in entry:
+            seen += 1
+            n = int(m.group(1))
+            if n != PREFILL_LAUNCH_REGS:
+                raise RuntimeError(f"{entry}: launches with {n} registers, the setmaxnreg split needs "
+                                   f"{PREFILL_LAUNCH_REGS}")
+            entry = None
+    if seen == 0:
+        raise RuntimeError("ptxas reported no prefill kernel register counts")
+
+
+def build(verbose: bool = False, force: bool = False, defines=(), out: str = None) -> str:
+    """Compiles the library.  ``defines`` (e.g. ``["ATTN_EMU_PAIRS_PER8=3"]``)
+    and ``out`` build a variant at another path; the default build needs
+    neither."""
+    out = out or LIB_PATH
+    if not force and not defines and out == LIB_PATH and up_to_date():
         return LIB_PATH
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include")]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    tmp = LIB_PATH + ".tmp"
+    cmd += [f"-D{d}" for d in defines]
+    cmd += ["-Xptxas", "-v"]
+    tmp = out + ".tmp"
     cmd += ["-o", tmp, *sources()]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    try:
+        check_register_counts(res.stdout + res.stderr)
+    except RuntimeError:
+        os.unlink(tmp)
+        raise
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-D", dest="defines", action="append", default=[])
+    ap.add_argument("--out", default=None)
+    a = ap.parse_args()
+    print(build(verbose=a.verbose, force=a.force, defines=a.defines, out=a.out))

@@ -2,6 +2,7 @@
 // CUDA call), the per-device status word, debug switches, and dispatch to the
 // kernel launchers.
 #include <atomic>
+#include <cstdio>
 #include <cstdint>
 #include <mutex>
 
@@ -35,6 +36,15 @@ int* device_status_word() {
     g_status_ptr[dev] = static_cast<int*>(ptr);
   }
   return g_status_ptr[dev];
+}
+
+namespace {
+thread_local char g_msg[256] = "";
+}
+
+int fail_cuda(const char* where, cudaError_t err) {
+  snprintf(g_msg, sizeof(g_msg), "%s: %s", where, cudaGetErrorString(err));
+  return ATTN_ERR_CUDA;
 }
 
 int debug_flags() { return g_debug_flags.load(); }
@@ -161,3 +171,5 @@ ATTN_API int attn_set_debug(int flags, unsigned long long wait_timeout_ns) {
 }
 
 ATTN_API int attn_version(void) { return 1; }
+
+ATTN_API const char* attn_last_error_message(void) { return g_msg; }

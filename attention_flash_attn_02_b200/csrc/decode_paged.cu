@@ -173,9 +173,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
   float l_part[2] = {0.f, 0.f}, r_part[2] = {0.f, 0.f};
   const float sl2 = p.scale_log2;
 
+  const int mi = lane >> 3, rr = lane & 7;
+  uint32_t qa[kD / 16][4];  // A fragments of this warp's 16 query rows, loaded once
   for (int ch = 0; ch < nchunks; ++ch) {
     cp_async_wait<kStages - 2>();
     __syncthreads();
+    if (ch == 0) {
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk)
+        ldsm_x4(s_q + swz(mt * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)), qa[kk][0], qa[kk][1], qa[kk][2],
+                qa[kk][3]);
+    }
     if (ch + kStages - 1 < nchunks) load_chunk(ch + kStages - 1, (ch + kStages - 1) % kStages);
     cp_async_commit();
     const uint32_t sk = s_kv + (ch % kStages) * 2 * kTileBytes;
@@ -185,15 +193,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
     float s[2][4];
 #pragma unroll
     for (int n = 0; n < 2; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-    const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
     for (int kk = 0; kk < kD / 16; ++kk) {
-      uint32_t a[4];
-      ldsm_x4(s_q + swz(mt * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)), a[0], a[1], a[2], a[3]);
       uint32_t b0, b1, b2, b3;
       ldsm_x4(sk + swz(sub * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)), b0, b1, b2, b3);
-      mma_bf16(s[0], a, b0, b1);
-      mma_bf16(s[1], a, b2, b3);
+      mma_bf16(s[0], qa[kk], b0, b1);
+      mma_bf16(s[1], qa[kk], b2, b3);
     }
     // mask tokens past the end of this split
     const int base_tok = ch * kChunk + sub * 16 + (lane & 3) * 2;
@@ -263,8 +268,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
   __syncthreads();  // stages are free: reuse them for the merge
 
   // Merge the 4 token slices of each query tile through shared memory.
-  float* s_o = reinterpret_cast<float*>(smem + kQBytes);        // [8 warps][16 rows][128]
-  float* s_ml = s_o + 8 * 16 * kD;                              // [8 warps][16 rows][3]
+  constexpr int kOS = kD + 4;  // padded row stride of the merge buffer (bank spread)
+  float* s_o = reinterpret_cast<float*>(smem + kQBytes);        // [8 warps][16 rows][kOS]
+  float* s_ml = s_o + 8 * 16 * kOS;                             // [8 warps][16 rows][3]
   {
     const int r0 = lane >> 2;
 #pragma unroll
@@ -283,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
       const int col = n * 8 + (lane & 3) * 2;
-      *reinterpret_cast<float2*>(&s_o[(warp * 16 + r0) * kD + col]) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(&s_o[(warp * 16 + r0 + 8) * kD + col]) = make_float2(o[n][2], o[n][3]);
+      *reinterpret_cast<float2*>(&s_o[(warp * 16 + r0) * kOS + col]) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(&s_o[(warp * 16 + r0 + 8) * kOS + col]) = make_float2(o[n][2], o[n][3]);
     }
   }
   __syncthreads();
@@ -314,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int sb = 0; sb < 4; ++sb) {
-          const float4 v = *reinterpret_cast<const float4*>(&s_o[((sb * 2 + mtile) * 16 + r) * kD + c0 + c]);
+          const float4 v = *reinterpret_cast<const float4*>(&s_o[((sb * 2 + mtile) * 16 + r) * kOS + c0 + c]);
           acc.x += w[sb] * v.x;
           acc.y += w[sb] * v.y;
           acc.z += w[sb] * v.z;
@@ -347,20 +353,53 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   const int nsplit = ((len + kPage - 1) / kPage + kDecodePagesPerSplit - 1) / kDecodePagesPerSplit;
   const float* base_o = p.ws_o + (size_t)gw * p.max_splits * kD;
   const float* base_l = p.ws_lse + (size_t)gw * p.max_splits;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base_l[s]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float L = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float l2 = base_l[s];
-      const float w = (l2 == -INFINITY) ? 0.f : ex2_approx(l2 - M);
-      const float4 v = *reinterpret_cast<const float4*>(base_o + (size_t)s * kD + lane * 4);
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
-      L += w;
+  float M = -INFINITY, L = 0.f;
+  // splits in groups of 32: lane s owns split s of the group
+  for (int s0 = 0; s0 < nsplit; s0 += 32) {
+    const int n = min(32, nsplit - s0);
+    const float l2 = lane < n ? base_l[s0 + lane] : -INFINITY;
+    float gm = l2;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+    const float Mn = fmaxf(M, gm);
+    if (Mn == -INFINITY) continue;
+    const float scale_old = (M == -INFINITY) ? 0.f : ex2_approx(M - Mn);
+    acc.x *= scale_old;
+    acc.y *= scale_old;
+    acc.z *= scale_old;
+    acc.w *= scale_old;
+    L *= scale_old;
+    M = Mn;
+    const float w = (l2 == -INFINITY) ? 0.f : ex2_approx(l2 - M);
+    float ws = w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+    L += ws;
+    int s = 0;
+    for (; s + 4 <= n; s += 4) {  // four independent loads in flight
+      float4 v[4];
+      float wv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[u] = *reinterpret_cast<const float4*>(base_o + (size_t)(s0 + s + u) * kD + lane * 4);
+        wv[u] = __shfl_sync(0xffffffffu, w, s + u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc.x += wv[u] * v[u].x;
+        acc.y += wv[u] * v[u].y;
+        acc.z += wv[u] * v[u].z;
+        acc.w += wv[u] * v[u].w;
+      }
+    }
+    for (; s < n; ++s) {
+      const float4 v = *reinterpret_cast<const float4*>(base_o + (size_t)(s0 + s) * kD + lane * 4);
+      const float wv = __shfl_sync(0xffffffffu, w, s);
+      acc.x += wv * v.x;
+      acc.y += wv * v.y;
+      acc.z += wv * v.z;
+      acc.w += wv * v.w;
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -380,11 +419,11 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int max_splits = decode_max_splits(a.max_pages);
   static bool attr_set[64] = {false};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -3;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
-      return -3;
+    err = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return fail_cuda("decode: cudaFuncSetAttribute", err);
     attr_set[dev] = true;
   }
   SplitParams sp{};
@@ -405,10 +444,11 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   sp.scale_log2 = a.scale * kLog2e;
   sp.bounds_check = (debug_flags() & 1) ? 1 : 0;
   sp.status = device_status_word();
-  if (!sp.status) return -3;
+  if (!sp.status) return fail_cuda("decode: status word", cudaGetLastError());
   dim3 grid(max_splits, a.B * a.Hkv);
   decode_split_kernel<<<grid, kThreads, kSmemBytes, stream>>>(sp);
-  if (cudaGetLastError() != cudaSuccess) return -3;
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail_cuda("decode: split launch", err);
   CombineParams cp{};
   cp.ws_o = sp.ws_o;
   cp.ws_lse = sp.ws_lse;
@@ -421,7 +461,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cp.max_splits = max_splits;
   const int nw = a.B * a.Hq;
   decode_combine_kernel<<<(nw + 7) / 8, 256, 0, stream>>>(cp);
-  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+  err = cudaGetLastError();
+  return err == cudaSuccess ? 0 : fail_cuda("decode: combine launch", err);
 }
 
 }  // namespace attn

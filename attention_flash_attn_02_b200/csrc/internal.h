@@ -43,12 +43,18 @@ unsigned long long wait_timeout_ns();
 // Number of SMs of the current device (cached).
 int sm_count();
 
+// Records a host-side failure for attn_last_error_message(); returns -3.
+int fail_cuda(const char* where, cudaError_t err);
+
 // Launchers: return a status code of include/attn.h.
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
 // Decode work split (shared by the workspace-size query and the launcher).
-constexpr int kDecodePagesPerSplit = 32;  // 512 tokens per split CTA
+#ifndef ATTN_DECODE_PAGES_PER_SPLIT
+#define ATTN_DECODE_PAGES_PER_SPLIT 32
+#endif
+constexpr int kDecodePagesPerSplit = ATTN_DECODE_PAGES_PER_SPLIT;  // 512 tokens per split CTA
 inline int decode_max_splits(int max_pages) {
   return (max_pages + kDecodePagesPerSplit - 1) / kDecodePagesPerSplit;
 }

@@ -10,11 +10,12 @@
 // blocks wholly above the causal diagonal or before the sliding window are
 // never loaded (kler.cn page §一.2; window of the zeeklog page).
 //
-// B200 mapping (one persistent CTA per SM, 320 threads):
+// B200 mapping (one persistent CTA per SM, 384 threads):
 //   warps 0-3   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 4-7   softmax warpgroup for Q tile 1
 //   warp  8     TMA producer: Q tiles, then K_j, V_j into a ring of stages
 //   warp  9     MMA issuer (one thread) + TMEM owner
+//   warps 10-11 idle (complete the third warpgroup)
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,..).
 // P (bf16 or e4m3) is written back over the first columns of its S buffer
 // and consumed from TMEM as the A operand of O += P V.
@@ -42,9 +43,25 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per K/V block
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // 3 warpgroups
+// Register split (setmaxnreg): the block launches with kLaunchRegs per thread
+// (384 threads x 168 fills the register file: 3 warps per SM sub-partition).
+// The producer/MMA warpgroup gives registers back and the two softmax
+// warpgroups take them.  The shares must add up to exactly the launch total
+// or the increase would wait forever: 2 * 200 + 104 = 3 * 168.  The build
+// checks with ptxas that the kernels launch with kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kOtherRegs = 104;
+static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must match the launch total");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
+// Of every 8 pairs of exponentials, this many are computed by the FMA-pipe
+// polynomial instead of the MUFU ex2 unit (balances the two pipes).
+#ifndef ATTN_EMU_PAIRS_PER8
+#define ATTN_EMU_PAIRS_PER8 2
+#endif
+constexpr int kEmuPairsPer8 = ATTN_EMU_PAIRS_PER8;
 
 template <int D, bool FP8>
 struct Cfg {
@@ -54,17 +71,21 @@ struct Cfg {
   static constexpr int BOX_ELEMS = 128 / EL;             // elements per box row
   static constexpr int BOX_BYTES = kBM * 128;            // one box: 128 rows x 128 B
   static constexpr int TILE_BYTES = kBM * ROW_BYTES;
-  static constexpr int NS = TILE_BYTES >= 32768 ? 4 : 8;  // K/V ring stages
+#ifndef ATTN_KV_STAGES_BIG
+#define ATTN_KV_STAGES_BIG 5
+#define ATTN_KV_STAGES_SMALL 12
+#endif
+  static constexpr int NS = TILE_BYTES >= 32768 ? ATTN_KV_STAGES_BIG : ATTN_KV_STAGES_SMALL;  // K/V ring stages
   static constexpr int MMA_K = FP8 ? 32 : 16;
   static constexpr int S_KSTEPS = D / MMA_K;
   static constexpr int PV_KSTEPS = kBN / MMA_K;
-  static constexpr int P_COLS = kBN * EL / 4;             // TMEM columns holding P
   static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
   static constexpr uint32_t IDESC_S = make_idesc(FP8 ? 0u : 1u, kBM, kBN, false);
   static constexpr uint32_t IDESC_PV = make_idesc(FP8 ? 0u : 1u, kBM, D, true);
   // shared memory: [Q0][Q1][stage 0..NS-1] (1024-aligned) + barriers
   static constexpr int SMEM_TILES = (2 + NS) * TILE_BYTES;
-  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align slack*/ + 256 /*barriers*/;
+  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align slack*/ + 512 /*barriers*/;
+  static_assert(SMEM_BYTES <= 232448, "more than the 227 KB a CTA may use");
   static_assert(NBOX >= 1 && ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle rows");
   static_assert(TM_O1 + D <= 512, "TMEM budget");
 };
@@ -108,7 +129,9 @@ __device__ __forceinline__ void key_range(int i, const Params& p, int& lo, int& 
 }
 
 // Units are numbered so that the longest (latest rows under a causal mask)
-// come first; CTA c takes units c, c + grid, ...
+// come first.  CTA c takes one unit per round, in snake order (c in even
+// rounds, grid - 1 - c in odd rounds), which balances the causal work across
+// CTAs to within a fraction of a percent without any global queue.
 __device__ __forceinline__ Unit get_unit(int u, const Params& p) {
   Unit w;
   const int mg = p.n_mgroups - 1 - u / p.n_pairs;
@@ -151,15 +174,27 @@ __device__ __forceinline__ Unit get_unit(int u, const Params& p) {
   return w;
 }
 
+__device__ __forceinline__ int unit_of(int round, int n_units) {
+  const int g = (int)gridDim.x, c = (int)blockIdx.x;
+#ifdef ATTN_ROUND_ROBIN
+  const int u = round * g + c;
+#else
+  const int u = round * g + ((round & 1) ? g - 1 - c : c);
+#endif
+  return u < n_units ? u : n_units;  // n_units: no more work
+}
+
 struct Smem {
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], p_full[2];
   uint64_t o_full[2], o_empty[2];
   uint64_t drain;
-  uint64_t kv_full[8], kv_empty[8];
+  uint64_t kv_full[12], kv_empty[12];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(Smem) <= 512, "barrier block exceeds its reserve");
 
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -210,12 +245,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitGuard g{&sm.abort_flag, p.status, p.timeout_ns, true};
   const WaitGuard g_drain{&sm.abort_flag, p.status, p.timeout_ns, false};
 
-  if (warp == 8) {
+  // Teardown, run at the end of every role branch (no code is shared between
+  // the register regions set by setmaxnreg): all threads meet, then the
+  // owner warp releases TMEM.
+  auto finish = [&]() {
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+    if (warp == 9) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+  };
+
+  if (warp >= 8) {
+    // Third warpgroup: hand registers back to the softmax warpgroups.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+  }
+  if (warp >= 10) {
+    // spare warps of the third warpgroup
+    finish();
+  } else if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t seq = 0, nunit = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
         const Unit w = get_unit(u, p);
         if (w.nb <= 0) continue;
         for (int t = 0; t < 2 && ok; ++t) {
@@ -253,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nunit > 0)
         for (int t = 0; t < 2; ++t) mbar_wait(&sm.q_full[t], (nunit - 1) & 1, g_drain);
     }
+    finish();
   } else if (warp == 9) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -284,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ts(tO[t], a, b, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
         const Unit w = get_unit(u, p);
         if (w.nb <= 0) continue;
         ok = mbar_wait(&sm.q_full[0], nunit & 1, g) && mbar_wait(&sm.q_full[1], nunit & 1, g);
@@ -345,8 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.drain, 0, g_drain);
     }
     __syncwarp();
+    finish();
   } else {
     // ------------------------------------------------------------ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     const int t = warp >> 2;                 // tile of this warpgroup
     const int r = ((warp & 3) << 5) + lane;  // row within the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
@@ -355,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t scnt = 0, nunit = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
       const Unit w = get_unit(u, p);
       const int row = w.m0[t] + r;
       const bool row_valid = row < p.Lq;
@@ -370,25 +427,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           ++scnt;
           tc_fence_after();
-          float s[kBN];
-#pragma unroll
-          for (int c = 0; c < kBN / 32; ++c) {
-            uint32_t raw[32];
-            tmem_ld32(tS + c * 32, raw);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[i]);
-          }
+          uint32_t sr[kBN];  // raw fp32 scores of this row
+          tmem_ld128(tS, sr);
           const int key0 = (w.kb_lo + j) * kBN;
-          if (!(lo <= key0 && key0 + kBN <= hi)) {
+          if (!(lo <= key0 && key0 + kBN <= hi)) {  // diagonal / window-edge / ragged block
 #pragma unroll
             for (int c = 0; c < kBN; ++c) {
               const int key = key0 + c;
-              if (key < lo || key >= hi) s[c] = -INFINITY;
+              if (key < lo || key >= hi) sr[c] = 0xFF800000u;  // -inf
             }
           }
-          float mx = s[0];
+          // row max: 8 independent partial maxima, 3-input max
+          float pm[8];
 #pragma unroll
-          for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+          for (int i = 0; i < 8; ++i) pm[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
+#pragma unroll
+          for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pm[i] = max3(pm[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+          const float mx = fmaxf(max3(pm[0], pm[1], pm[2]), max3(max3(pm[3], pm[4], pm[5]), pm[6], pm[7]));
           const float m_blk = mx * sl2;
           float alpha = 1.f;
           if (m_blk > m_run + kRescaleThreshold) {
@@ -398,38 +456,56 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run *= alpha;
           l_rnd *= alpha;
           const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-          float rs = 0.f, rr = 0.f;
-          if (FP8) {
-            uint32_t pk[32];
+          const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
+          // P = 2^(s * scale * log2e - m); exact and rounded row sums in four
+          // independent packed accumulators each.
+          uint64_t rs2[4] = {0, 0, 0, 0}, rr2[4] = {0, 0, 0, 0};
+          uint32_t pk[kBN / 2];
 #pragma unroll
-            for (int c = 0; c < kBN; c += 4) {
-              const float p0 = ex2_approx(fmaf(s[c + 0], sl2, neg_m));
-              const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg_m));
-              const float p2 = ex2_approx(fmaf(s[c + 2], sl2, neg_m));
-              const float p3 = ex2_approx(fmaf(s[c + 3], sl2, neg_m));
-              const uint16_t lo = pack_e4m3x2(p0, p1), hi = pack_e4m3x2(p2, p3);
-              pk[c / 4] = (uint32_t)lo | ((uint32_t)hi << 16);
-              rs += (p0 + p1) + (p2 + p3);
-              rr += sum_e4m3x4(lo, hi);
+          for (int q2 = 0; q2 < kBN / 2; ++q2) {
+            const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
+            float p0, p1;
+            if ((q2 & 7) >= 8 - kEmuPairsPer8) {
+              f2_split(exp2_poly2(x2), p0, p1);
+            } else {
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
             }
-            tmem_st32(tS, pk);
-          } else {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t pk[32];
-#pragma unroll
-              for (int c = 0; c < 64; c += 2) {
-                const float p0 = ex2_approx(fmaf(s[h * 64 + c], sl2, neg_m));
-                const float p1 = ex2_approx(fmaf(s[h * 64 + c + 1], sl2, neg_m));
-                pk[c / 2] = pack_bf16x2(p0, p1);
-                rs += p0 + p1;
-                rr += sum_bf16x2(pk[c / 2]);
-              }
-              tmem_st32(tS + h * 32, pk);
+            rs2[q2 & 3] = add2(rs2[q2 & 3], f2(p0, p1));
+            if (FP8) {
+              const uint16_t e = pack_e4m3x2(p0, p1);
+              if (q2 & 1) pk[q2 >> 1] |= (uint32_t)e << 16;
+              else pk[q2 >> 1] = e;
+              uint32_t h;
+              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(e));
+              float h0, h1;
+              asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+                  : "=f"(h0), "=f"(h1)
+                  : "r"(h));
+              rr2[q2 & 3] = add2(rr2[q2 & 3], f2(h0, h1));
+            } else {
+              const uint32_t b = pack_bf16x2(p0, p1);
+              pk[q2] = b;
+              rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
             }
           }
-          l_run += rs;
-          l_rnd += rr;
+          if (FP8) {
+            tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+          } else {
+            tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+            tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+          }
+          {
+            const uint64_t a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
+            const uint64_t b = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
+            float a0, a1, b0, b1;
+            f2_split(a, a0, a1);
+            f2_split(b, b0, b1);
+            l_run += a0 + a1;
+            l_rnd += b0 + b1;
+          }
           // Rescale the accumulator when the running max moved.  The previous
           // P.V of this tile has completed: it was issued before this S.
           const bool need = (j > 0) && (alpha != 1.f);
@@ -482,13 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++nunit;
       }
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    finish();
   }
 }
 
@@ -526,11 +596,11 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   using C = Cfg<D, FP8>;
   static bool attr_set[64] = {false};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -3;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(prefill_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return -3;
+    err = cudaFuncSetAttribute(prefill_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (err != cudaSuccess) return fail_cuda("prefill: cudaFuncSetAttribute", err);
     attr_set[dev] = true;
   }
   Params p{};
@@ -557,20 +627,21 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * log2e * (FP8 ? a.q_descale * a.k_descale : 1.f);
   p.out_scale = FP8 ? a.v_descale : 1.f;
   p.status = device_status_word();
-  if (!p.status) return -3;
+  if (!p.status) return fail_cuda("prefill: status word", cudaGetLastError());
   p.timeout_ns = wait_timeout_ns();
 
   CUtensorMap tq, tk, tv;
   const bool have_k = a.Lk > 0;
-  if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq)) return -3;
+  if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq)) return fail_cuda("prefill: tensor map (q)", cudaErrorInvalidValue);
   // With no keys nothing is loaded from K/V; describe Q instead of an empty tensor.
   if (!encode_3d(&tk, have_k ? a.k : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
-    return -3;
+    return fail_cuda("prefill: tensor map (k)", cudaErrorInvalidValue);
   if (!encode_3d(&tv, have_k ? a.v : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
-    return -3;
+    return fail_cuda("prefill: tensor map (v)", cudaErrorInvalidValue);
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
   prefill_kernel<D, FP8><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+  err = cudaGetLastError();
+  return err == cudaSuccess ? 0 : fail_cuda("prefill: launch", err);
 }
 
 }  // namespace

@@ -131,9 +131,14 @@ class ClockSampler:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 9:
                 rows.append(parts)
-        uuids = {r[0].lower() for r in rows}
-        mine = [r for r in rows if self.uuid and self.uuid in r[0].lower()]
+        norm = lambda u: u.lower().replace("gpu-", "").replace("-", "")  # noqa: E731
+        uuids = {norm(r[0]) for r in rows}
+        mine = [r for r in rows if self.uuid and norm(r[0]) == norm(self.uuid)]
+        seen = sorted(uuids)
         rows = mine if mine else (rows if len(uuids) == 1 else [])
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["device not matched"],
+                    "samples": 0, "uuid": self.uuid, "seen": seen[:8]}
         os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}

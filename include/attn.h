@@ -182,6 +182,13 @@ ATTN_API const char* attn_status_str(int status);
 #define ATTN_DEBUG_BOUNDS 1
 ATTN_API int attn_set_debug(int flags, unsigned long long wait_timeout_ns);
 
+/*
+ * attn_last_error_message -- static, human-readable description of the last
+ * host-side CUDA failure on the calling thread (the call that returned
+ * ATTN_ERR_CUDA and the CUDA error string); "" if none.
+ */
+ATTN_API const char* attn_last_error_message(void);
+
 /* attn_version -- ABI version of this header (currently 1). */
 ATTN_API int attn_version(void);
 
