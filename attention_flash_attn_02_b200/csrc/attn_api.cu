@@ -111,8 +111,7 @@ ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
 
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D) {
   if (B <= 0 || Hq <= 0 || max_pages_per_seq <= 0 || D <= 0) return 0;
-  // normalised partial outputs (D floats) and their log-sum-exp (1 float)
-  return (size_t)B * Hq * decode_max_splits(max_pages_per_seq) * (size_t)(D + 1) * sizeof(float);
+  return decode_workspace_bytes(B, Hq, max_pages_per_seq, D);
 }
 
 ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,

@@ -4,22 +4,28 @@
 // per-sequence block table), for B200 (sm_100a).
 //
 // Two launches:
-//   decode_split_kernel   grid (splits, B * Hkv).  Each CTA takes one K/V head
-//       of one sequence and a run of kPagesPerSplit pages (512 tokens), gathers
-//       the pages with 16-byte cp.async into swizzled shared memory (3-stage
-//       ring), and computes, for all Hq/Hkv query heads of the group at once,
-//       S = q K^T and O += P V on the tensor cores (mma.sync m16n8k16 bf16 ->
-//       fp32) with the online-softmax recurrence.  It writes one partial
-//       (normalised o, log2-sum-exp) per query head and split.
+//   decode_split_kernel   G = 3 CTAs per SM.  All cached pages of the batch,
+//       sequence after sequence (and K/V head after K/V head), form one list
+//       of T pages; CTA c streams the contiguous share [c T / G, (c+1) T / G)
+//       of it (at least kDecodeMinChunk pages), so every CTA moves the same
+//       number of bytes whatever the length mix.  Warp 2 is a TMA producer:
+//       it loads the 32 query rows of each sequence segment it meets and
+//       copies whole pages (K and V, 128-byte swizzled) straight from the pool
+//       into a 6-stage ring tracked by mbarriers.  Warps 0 and 1 take query
+//       rows [0, 16) and [16, 32) of the K/V group and compute S = q K^T and
+//       O += P V on the tensor cores (mma.sync m16n8k16 bf16 -> fp32) with the
+//       online-softmax recurrence; at the end of a segment they write one
+//       partial (normalised o, log2-sum-exp) per query head.
 //   decode_combine_kernel one warp per (sequence, query head) merges the
 //       partials: M = max_s lse_s, O = sum_s 2^(lse_s - M) o_s / sum_s
 //       2^(lse_s - M), LSE = (M + log2 sum) ln 2.  This is the rescaling step of
 //       the online softmax (page "003-注意力机制详解...", §二) applied once
-//       across splits.
+//       across segments.
 // All query heads of a K/V group share every gathered page (MQA/GQA: the
 // tqpw.cn article §2.1/§3.1), which is what makes the tensor cores necessary:
 // with 32 heads per K/V head, a SIMT dot product would be compute-bound.
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 #include <cstdint>
 
 #include "internal.h"
@@ -30,50 +36,108 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kPage = 16;
-constexpr int kThreads = 256;            // 8 warps
-constexpr int kChunk = 64;               // tokens per pipeline stage
-constexpr int kStages = 3;
-constexpr int kRowBytes = kD * 2;        // 256
-constexpr int kTileBytes = kChunk * kRowBytes;  // 16 KB (K or V of one stage)
-constexpr int kQBytes = 32 * kRowBytes;          // 32 query rows (8 KB)
-constexpr int kSmemBytes = kQBytes + kStages * 2 * kTileBytes + 256;
+constexpr int kThreads = 96;                 // 2 consumer warps + 1 producer warp
+#ifndef ATTN_DECODE_STAGES
+#define ATTN_DECODE_STAGES 6
+#define ATTN_DECODE_CTAS_PER_SM 3
+#endif
+constexpr int kStages = ATTN_DECODE_STAGES;
+constexpr int kCtasPerSm = ATTN_DECODE_CTAS_PER_SM;
+constexpr int kHalfBox = kPage * 128;        // 16 tokens x 64 features (bf16): 2 KB
+constexpr int kPageBytes = 2 * kHalfBox;     // K (or V) of one page: 4 KB
+constexpr int kStageBytes = 2 * kPageBytes;  // K and V of one page: 8 KB
+constexpr int kQRows = 32;                   // query rows per K/V group tile
+constexpr int kQBox = kQRows * 128;          // 32 rows x 64 features: 4 KB
+constexpr int kQBytes = 2 * kQBox;           // 8 KB per query slot
+constexpr int kRingOff = 2 * kQBytes;        // two query slots, then the ring
+constexpr int kSmemBytes = 1024 + kRingOff + kStages * kStageBytes + 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct SplitParams {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* k_pages;
-  const __nv_bfloat16* v_pages;
   const int* block_table;
   const int* seq_lens;
-  float* ws_o;    // [B * Hq][max_splits][kD] normalised partial outputs
-  float* ws_lse;  // [B * Hq][max_splits] log2-sum-exp of each partial
-  int B, Hq, Hkv, group, num_pages, max_pages, max_splits;
+  float* ws_o;    // [B * Hq][S][kD] normalised partial outputs
+  float* ws_lse;  // [B * Hq][S] log2-sum-exp of each partial
+  int* ws_nseg;   // [B * Hkv] segments of each (sequence, K/V head)
+  int B, Hq, Hkv, group, num_pages, max_pages, max_segs;
   float scale_log2;
   int bounds_check;
   int* status;
+  unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ int seq_len_of(const SplitParams& p, int b) {
-  int n = p.seq_lens[b];
-  const int cap = p.max_pages * kPage;
+struct DecSmem {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t qfull[2], qempty[2];
+  int valid[kStages];
+  int abort_flag;
+};
+static_assert(sizeof(DecSmem) <= 256, "barrier block exceeds its reserve");
+static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "CTAs per SM do not fit in shared memory");
+
+__device__ __forceinline__ int len_of(const int* seq_lens, int max_pages, int b) {
+  const int n = seq_lens[b], cap = max_pages * kPage;
   return n < 0 ? 0 : (n > cap ? cap : n);
 }
-
-// Byte offset of 16-byte chunk `c` of row `r` in a swizzled [rows][256 B] tile.
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-  return (uint32_t)(r * kRowBytes + ((c ^ (r & 7)) << 4));
+__device__ __forceinline__ int pages_of(const int* seq_lens, int max_pages, int b) {
+  return (len_of(seq_lens, max_pages, b) + kPage - 1) / kPage;
+}
+// CTA that owns page x of the list when T pages are split over G CTAs.
+__device__ __forceinline__ int owner(long long x, long long T, int G) {
+  return (int)(((x + 1) * G - 1) / T);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;  // 0: zero-fill, nothing read
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Walks the (sequence, K/V head) segments a CTA's page range [lo, hi) meets.
+struct Segments {
+  const SplitParams& p;
+  long long hi;
+  long long x;    // next page of the list
+  long long pre;  // list index of the first page of the current (b, kvh)
+  int b, kvh, P;  // current sequence, K/V head, its page count
+  __device__ Segments(const SplitParams& p_, long long lo, long long hi_) : p(p_), hi(hi_), x(lo) {
+    long long c = 0;
+    b = 0;
+    kvh = 0;
+    P = 0;
+    pre = 0;
+    for (; b < p.B; ++b) {
+      P = pages_of(p.seq_lens, p.max_pages, b);
+      if (lo < c + (long long)p.Hkv * P) {
+        kvh = (int)((lo - c) / P);
+        pre = c + (long long)kvh * P;
+        return;
+      }
+      c += (long long)p.Hkv * P;
+    }
+  }
+  __device__ bool more() const { return x < hi; }
+  // pages [pg_lo, pg_hi) of sequence b, K/V head kvh; then advances
+  __device__ void take(int& sb, int& skvh, int& pg_lo, int& pg_hi, long long& spre, int& sP) {
+    const long long end = pre + P < hi ? pre + P : hi;
+    sb = b;
+    skvh = kvh;
+    spre = pre;
+    sP = P;
+    pg_lo = (int)(x - pre);
+    pg_hi = (int)(end - pre);
+    x = end;
+    pre += P;
+    if (++kvh == p.Hkv) {
+      kvh = 0;
+      do {
+        ++b;
+        P = b < p.B ? pages_of(p.seq_lens, p.max_pages, b) : 1;
+      } while (b < p.B && P == 0);
+    }
+  }
+};
+
+// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled
+// TMA box (rows of 128 bytes, base 1024-aligned).
+__device__ __forceinline__ uint32_t sw128(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -96,182 +160,246 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int split = blockIdx.x;
-  const int bk = blockIdx.y;
-  const int b = bk / p.Hkv, kvh = bk % p.Hkv;
-  const int len = seq_len_of(p, b);
-  const int npages = (len + kPage - 1) / kPage;
-  const int pg0 = split * kDecodePagesPerSplit;
-  if (pg0 >= npages) return;
-  const int pg1 = min(pg0 + kDecodePagesPerSplit, npages);
-  const int tok0 = pg0 * kPage;
-  const int tok1 = min(pg1 * kPage, len);
-  const int ntok = tok1 - tok0;
-  const int nchunks = (ntok + kChunk - 1) / kChunk;
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // Total pages T of the batch and this CTA's share.
+  long long T = 0;
+  for (int b = 0; b < p.B; ++b) T += (long long)p.Hkv * pages_of(p.seq_lens, p.max_pages, b);
+  long long G = T / kDecodeMinChunk;
+  if (G > (long long)gridDim.x) G = gridDim.x;
+  if (G < 1) G = 1;
+  const int c = blockIdx.x;
+  if (T == 0 || c >= G) return;
+  const long long lo = c * T / G, hi = (c + 1) * T / G;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t s_q = smem_u32(smem);
-  const uint32_t s_kv = s_q + kQBytes;
-  int* s_pages = reinterpret_cast<int*>(smem + kQBytes + kStages * 2 * kTileBytes);
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t s_q = base;                // 2 query slots of 8 KB
+  const uint32_t s_ring = base + kRingOff;  // kStages x 8 KB
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(base_ptr + kRingOff + kStages * kStageBytes);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 2);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.qfull[s], 1);
+      mbar_init(&sm.qempty[s], 2);
+    }
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  const WaitGuard g{&sm.abort_flag, p.status, p.timeout_ns, true};
+  const WaitGuard g_drain{&sm.abort_flag, p.status, p.timeout_ns, false};
 
-  // Page ids of this split (bounds-checked on request).
-  if (tid < kDecodePagesPerSplit) {
-    int id = 0;
-    if (pg0 + tid < pg1) {
-      id = p.block_table[(size_t)b * p.max_pages + pg0 + tid];
-      if (p.bounds_check && (id < 0 || id >= p.num_pages)) {
-        atomicExch(p.status, kErrBounds);
-        id = -1;
+  if (warp == 2) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    uint32_t n_st = 0, n_q = 0;
+    bool ok = true;
+    Segments seg(p, lo, hi);
+    while (seg.more() && ok) {
+      int b, kvh, pg_lo, pg_hi, P;
+      long long pre;
+      seg.take(b, kvh, pg_lo, pg_hi, pre, P);
+      if (lane == 0) {  // query rows of this (sequence, K/V head)
+        const uint32_t qs = n_q & 1;
+        if (n_q >= 2) ok = mbar_wait(&sm.qempty[qs], ((n_q >> 1) - 1) & 1, g);
+        if (ok) {
+          mbar_arrive_expect_tx(&sm.qfull[qs], kQBytes);
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(s_q + qs * kQBytes + h * kQBox, &tm_q, &sm.qfull[qs], h * 64, b * p.Hq + kvh * p.group);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++n_q;
+      for (int k0 = pg_lo; k0 < pg_hi && ok; k0 += 32) {
+        // 32 page ids at a time, one per lane
+        int id = -1;
+        if (k0 + lane < pg_hi) {
+          id = p.block_table[(size_t)b * p.max_pages + k0 + lane];
+          if (p.bounds_check && (id < 0 || id >= p.num_pages)) {
+            atomicExch(p.status, kErrBounds);
+            id = -1;
+          }
+        }
+        const int kn = pg_hi - k0 < 32 ? pg_hi - k0 : 32;
+        for (int k = 0; k < kn && ok; ++k) {
+          const int pid = __shfl_sync(0xffffffffu, id, k);
+          if (lane == 0) {
+            const uint32_t st = n_st % kStages;
+            if (n_st >= (uint32_t)kStages) ok = mbar_wait(&sm.empty[st], ((n_st / kStages) - 1) & 1, g);
+            if (ok) {
+              sm.valid[st] = pid >= 0;
+              mbar_arrive_expect_tx(&sm.full[st], pid >= 0 ? kStageBytes : 0);
+              if (pid >= 0) {
+                const uint32_t dst = s_ring + st * kStageBytes;
+                for (int h = 0; h < 2; ++h) {
+                  tma_load_3d(dst + h * kHalfBox, &tm_k, &sm.full[st], h * 64, kvh, pid * kPage);
+                  tma_load_3d(dst + kPageBytes + h * kHalfBox, &tm_v, &sm.full[st], h * 64, kvh, pid * kPage);
+                }
+              }
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++n_st;
+        }
       }
     }
-    s_pages[tid] = id;
-  }
-  // Query rows of the group (rows >= group are zero).
-  {
-    const int row = tid >> 3;  // 32 rows x 16 chunks = 512 pieces, 2 per thread
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int c = (tid & 7) + 8 * i;
-      const bool valid = row < p.group;
-      const __nv_bfloat16* src = p.q + ((size_t)b * p.Hq + kvh * p.group + (valid ? row : 0)) * kD + c * 8;
-      cp_async16(s_q + swz(row, c), src, valid);
+    if (lane == 0) {
+      // Drain: the last loads of every slot have landed before the CTA exits.
+      for (uint32_t s = (n_st > (uint32_t)kStages ? n_st - kStages : 0); s < n_st; ++s)
+        mbar_wait(&sm.full[s % kStages], (s / kStages) & 1, g_drain);
+      for (uint32_t s = (n_q > 2u ? n_q - 2 : 0); s < n_q; ++s) mbar_wait(&sm.qfull[s & 1], (s >> 1) & 1, g_drain);
     }
-  }
-  __syncthreads();  // s_pages visible
-
-  auto load_chunk = [&](int ch, int stage) {
-    const uint32_t dk = s_kv + stage * 2 * kTileBytes;
-    const uint32_t dv = dk + kTileBytes;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int piece = tid + i * kThreads;  // 64 rows x 16 chunks
-      const int row = piece >> 4, c = piece & 15;
-      const int tok = ch * kChunk + row;      // token offset within the split
-      const int pid = s_pages[tok >> 4];
-      const bool valid = tok < ntok && pid >= 0;
-      const size_t off = valid ? ((((size_t)pid * kPage + (tok & 15)) * p.Hkv + kvh) * kD + c * 8) : 0;
-      cp_async16(dk + swz(row, c), p.k_pages + off, valid);
-      cp_async16(dv + swz(row, c), p.v_pages + off, valid);
-    }
-  };
-#pragma unroll
-  for (int st = 0; st < kStages - 1; ++st) {
-    if (st < nchunks) load_chunk(st, st);
-    cp_async_commit();  // group 0 also carries the query rows
+    return;
   }
 
-  const int mt = warp & 1;   // 16-row query tile
-  const int sub = warp >> 1; // 16-token slice of each chunk
-  float o[16][4];
-#pragma unroll
-  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  // per-lane partial row sums: exact fp32 (for the LSE) and of the rounded P
-  // the tensor cores multiply (normalises o)
-  float l_part[2] = {0.f, 0.f}, r_part[2] = {0.f, 0.f};
-  const float sl2 = p.scale_log2;
-
+  // -------------------------------------------------------------- consumers
+  const int mt = warp;  // query rows [16 mt, 16 mt + 16) of the group
   const int mi = lane >> 3, rr = lane & 7;
-  uint32_t qa[kD / 16][4];  // A fragments of this warp's 16 query rows, loaded once
-  for (int ch = 0; ch < nchunks; ++ch) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (ch == 0) {
+  const float sl2 = p.scale_log2;
+  uint32_t n_st = 0, n_q = 0;
+  bool ok = true;
+  Segments seg(p, lo, hi);
+  while (seg.more() && ok) {
+    int b, kvh, pg_lo, pg_hi, P;
+    long long pre;
+    seg.take(b, kvh, pg_lo, pg_hi, pre, P);
+    const int len = len_of(p.seq_lens, p.max_pages, b);
+    const uint32_t qs = n_q & 1;
+    ok = mbar_wait(&sm.qfull[qs], (n_q >> 1) & 1, g);
+    if (!ok) break;
+    ++n_q;
+    uint32_t qa[kD / 16][4];
 #pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk)
-        ldsm_x4(s_q + swz(mt * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)), qa[kk][0], qa[kk][1], qa[kk][2],
-                qa[kk][3]);
-    }
-    if (ch + kStages - 1 < nchunks) load_chunk(ch + kStages - 1, (ch + kStages - 1) % kStages);
-    cp_async_commit();
-    const uint32_t sk = s_kv + (ch % kStages) * 2 * kTileBytes;
-    const uint32_t sv = sk + kTileBytes;
+    for (int kk = 0; kk < kD / 16; ++kk)
+      ldsm_x4(s_q + qs * kQBytes + (kk >> 2) * kQBox + sw128(mt * 16 + (mi & 1) * 8 + rr, (kk & 3) * 2 + (mi >> 1)),
+              qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.qempty[qs]);  // query fragments are in registers
 
-    // S = q K^T for 16 query rows x 16 tokens
-    float s[2][4];
+    float o[16][4];
 #pragma unroll
-    for (int n = 0; n < 2; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(sk + swz(sub * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)), b0, b1, b2, b3);
-      mma_bf16(s[0], qa[kk], b0, b1);
-      mma_bf16(s[1], qa[kk], b2, b3);
-    }
-    // mask tokens past the end of this split
-    const int base_tok = ch * kChunk + sub * 16 + (lane & 3) * 2;
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tok = base_tok + n * 8 + (e & 1);
-        s[n][e] = tok < ntok ? s[n][e] * sl2 : -INFINITY;
-      }
-    // online softmax for rows r (e = 0,1) and r + 8 (e = 2,3)
-    float alpha[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float mx = fmaxf(fmaxf(s[0][2 * h], s[0][2 * h + 1]), fmaxf(s[1][2 * h], s[1][2 * h + 1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      alpha[h] = 1.f;
-      if (mx > m_run[h] + kRescaleThreshold) {
-        alpha[h] = ex2_approx(m_run[h] - mx);
-        m_run[h] = mx;
-      }
-      l_part[h] *= alpha[h];
-      r_part[h] *= alpha[h];
-    }
-    if (alpha[0] != 1.f || alpha[1] != 1.f) {
-#pragma unroll
-      for (int n = 0; n < 16; ++n) {
-        o[n][0] *= alpha[0];
-        o[n][1] *= alpha[0];
-        o[n][2] *= alpha[1];
-        o[n][3] *= alpha[1];
-      }
-    }
-    uint32_t pa[4];
-    {
-      const float nm0 = m_run[0] == -INFINITY ? 0.f : -m_run[0];
-      const float nm1 = m_run[1] == -INFINITY ? 0.f : -m_run[1];
-      float pv[2][4];
-#pragma unroll
-      for (int n = 0; n < 2; ++n) {
-        pv[n][0] = ex2_approx(s[n][0] + nm0);
-        pv[n][1] = ex2_approx(s[n][1] + nm0);
-        pv[n][2] = ex2_approx(s[n][2] + nm1);
-        pv[n][3] = ex2_approx(s[n][3] + nm1);
-        l_part[0] += pv[n][0] + pv[n][1];
-        l_part[1] += pv[n][2] + pv[n][3];
-      }
-      pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
-      pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
-      pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
-      pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
-      // row sums of the same rounded P the tensor cores multiply
-      r_part[0] += sum_bf16x2(pa[0]) + sum_bf16x2(pa[2]);
-      r_part[1] += sum_bf16x2(pa[1]) + sum_bf16x2(pa[3]);
-    }
-    // O += P V over 16 tokens x 128 features
-#pragma unroll
-    for (int n = 0; n < 16; n += 2) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(sv + swz(sub * 16 + (mi & 1) * 8 + rr, n + (mi >> 1)), b0, b1, b2, b3);
-      mma_bf16(o[n], pa, b0, b1);
-      mma_bf16(o[n + 1], pa, b2, b3);
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();  // stages are free: reuse them for the merge
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    // per-lane partial row sums: exact fp32 (for the LSE) and of the rounded
+    // P the tensor cores multiply (normalises o)
+    float l_part[2] = {0.f, 0.f}, r_part[2] = {0.f, 0.f};
 
-  // Merge the 4 token slices of each query tile through shared memory.
-  constexpr int kOS = kD + 4;  // padded row stride of the merge buffer (bank spread)
-  float* s_o = reinterpret_cast<float*>(smem + kQBytes);        // [8 warps][16 rows][kOS]
-  float* s_ml = s_o + 8 * 16 * kOS;                             // [8 warps][16 rows][3]
-  {
+    for (int k = pg_lo; k < pg_hi; ++k) {
+      const uint32_t st = n_st % kStages;
+      ok = mbar_wait(&sm.full[st], (n_st / kStages) & 1, g);
+      if (!ok) break;
+      ++n_st;
+      if (sm.valid[st]) {
+        const uint32_t sk = s_ring + st * kStageBytes;
+        const uint32_t sv = sk + kPageBytes;
+        // S = q K^T for 16 query rows x 16 tokens; even and odd k-steps in
+        // separate accumulators (two independent MMA chains)
+        float s[2][4], s2[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] = s2[n][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sk + (kk >> 2) * kHalfBox + sw128((mi >> 1) * 8 + rr, (kk & 3) * 2 + (mi & 1)), b0, b1, b2, b3);
+          if (kk & 1) {
+            mma_bf16(s2[0], qa[kk], b0, b1);
+            mma_bf16(s2[1], qa[kk], b2, b3);
+          } else {
+            mma_bf16(s[0], qa[kk], b0, b1);
+            mma_bf16(s[1], qa[kk], b2, b3);
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
+        // mask tokens past the end of the sequence
+        const int base_tok = k * kPage + (lane & 3) * 2;
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = base_tok + n * 8 + (e & 1);
+            s[n][e] = tok < len ? s[n][e] * sl2 : -INFINITY;
+          }
+        // online softmax for rows r (e = 0,1) and r + 8 (e = 2,3)
+        float alpha[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float mx = fmaxf(fmaxf(s[0][2 * h], s[0][2 * h + 1]), fmaxf(s[1][2 * h], s[1][2 * h + 1]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          alpha[h] = 1.f;
+          if (mx > m_run[h] + kRescaleThreshold) {
+            alpha[h] = ex2_approx(m_run[h] - mx);
+            m_run[h] = mx;
+          }
+          l_part[h] *= alpha[h];
+          r_part[h] *= alpha[h];
+        }
+        if (alpha[0] != 1.f || alpha[1] != 1.f) {
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            o[n][0] *= alpha[0];
+            o[n][1] *= alpha[0];
+            o[n][2] *= alpha[1];
+            o[n][3] *= alpha[1];
+          }
+        }
+        uint32_t pa[4];
+        {
+          const float nm0 = m_run[0] == -INFINITY ? 0.f : -m_run[0];
+          const float nm1 = m_run[1] == -INFINITY ? 0.f : -m_run[1];
+          float pv[2][4];
+#pragma unroll
+          for (int n = 0; n < 2; ++n) {
+            pv[n][0] = ex2_approx(s[n][0] + nm0);
+            pv[n][1] = ex2_approx(s[n][1] + nm0);
+            pv[n][2] = ex2_approx(s[n][2] + nm1);
+            pv[n][3] = ex2_approx(s[n][3] + nm1);
+            l_part[0] += pv[n][0] + pv[n][1];
+            l_part[1] += pv[n][2] + pv[n][3];
+          }
+          pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
+          pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
+          pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
+          pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
+          r_part[0] += sum_bf16x2(pa[0]) + sum_bf16x2(pa[2]);
+          r_part[1] += sum_bf16x2(pa[1]) + sum_bf16x2(pa[3]);
+        }
+        // O += P V over 16 tokens x 128 features
+#pragma unroll
+        for (int n = 0; n < 16; n += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(sv + (n >> 3) * kHalfBox + sw128((mi & 1) * 8 + rr, (n & 7) + (mi >> 1)), b0, b1, b2, b3);
+          mma_bf16(o[n], pa, b0, b1);
+          mma_bf16(o[n + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[st]);
+    }
+    if (!ok) break;
+    // One partial per query row of this warp for this segment.
+    const int sidx = c - owner(pre, T, (int)G);
+    if (sidx < 0 || sidx >= p.max_segs) {  // cannot happen with chunks >= kDecodeMinChunk pages
+      if (lane == 0) atomicExch(p.status, kErrBounds);
+      continue;
+    }
     const int r0 = lane >> 2;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -280,84 +408,48 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitPa
       l += __shfl_xor_sync(0xffffffffu, l, 2);
       lr += __shfl_xor_sync(0xffffffffu, lr, 1);
       lr += __shfl_xor_sync(0xffffffffu, lr, 2);
-      if ((lane & 3) == 0) {
-        s_ml[(warp * 16 + r0 + 8 * h) * 3 + 0] = m_run[h];
-        s_ml[(warp * 16 + r0 + 8 * h) * 3 + 1] = l;
-        s_ml[(warp * 16 + r0 + 8 * h) * 3 + 2] = lr;
+      const int row = mt * 16 + r0 + 8 * h;
+      if (row < p.group) {
+        const size_t rec = ((size_t)b * p.Hq + kvh * p.group + row) * p.max_segs + sidx;
+        const float inv = lr > 0.f ? 1.f / lr : 0.f;
+        float* dst = p.ws_o + rec * kD + (lane & 3) * 2;
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+          *reinterpret_cast<float2*>(dst + n * 8) = make_float2(o[n][2 * h] * inv, o[n][2 * h + 1] * inv);
+        if ((lane & 3) == 0) p.ws_lse[rec] = l > 0.f ? m_run[h] + __log2f(l) : -INFINITY;
       }
     }
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const int col = n * 8 + (lane & 3) * 2;
-      *reinterpret_cast<float2*>(&s_o[(warp * 16 + r0) * kOS + col]) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(&s_o[(warp * 16 + r0 + 8) * kOS + col]) = make_float2(o[n][2], o[n][3]);
-    }
-  }
-  __syncthreads();
-  // 32 rows x 128 features; each thread owns one row and 16 features.
-  {
-    const int row = tid >> 3;       // query row within the group tile (0..31)
-    const int c0 = (tid & 7) * 16;  // first feature
-    if (row < p.group) {
-      const int mtile = row >> 4, r = row & 15;
-      float M = -INFINITY;
-#pragma unroll
-      for (int sb = 0; sb < 4; ++sb) M = fmaxf(M, s_ml[((sb * 2 + mtile) * 16 + r) * 3]);
-      float w[4], L = 0.f, LR = 0.f;
-#pragma unroll
-      for (int sb = 0; sb < 4; ++sb) {
-        const float m = s_ml[((sb * 2 + mtile) * 16 + r) * 3];
-        w[sb] = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-        L += w[sb] * s_ml[((sb * 2 + mtile) * 16 + r) * 3 + 1];
-        LR += w[sb] * s_ml[((sb * 2 + mtile) * 16 + r) * 3 + 2];
-      }
-      const float inv = LR > 0.f ? 1.f / LR : 0.f;
-      const int h = kvh * p.group + row;
-      const size_t rec = ((size_t)b * p.Hq + h) * p.max_splits + split;
-      float* dst = p.ws_o + rec * kD;
-#pragma unroll
-      for (int c = 0; c < 16; c += 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int sb = 0; sb < 4; ++sb) {
-          const float4 v = *reinterpret_cast<const float4*>(&s_o[((sb * 2 + mtile) * 16 + r) * kOS + c0 + c]);
-          acc.x += w[sb] * v.x;
-          acc.y += w[sb] * v.y;
-          acc.z += w[sb] * v.z;
-          acc.w += w[sb] * v.w;
-        }
-        *reinterpret_cast<float4*>(dst + c0 + c) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      }
-      if (c0 == 0) p.ws_lse[rec] = (L > 0.f) ? M + __log2f(L) : -INFINITY;
-    }
+    if (sidx == 0 && mt == 0 && lane == 0)
+      p.ws_nseg[b * p.Hkv + kvh] = owner(pre + P - 1, T, (int)G) - owner(pre, T, (int)G) + 1;
   }
 }
 
 struct CombineParams {
   const float* ws_o;
   const float* ws_lse;
+  const int* ws_nseg;
   const int* seq_lens;
   __nv_bfloat16* o;
   float* lse;
-  int B, Hq, max_pages, max_splits;
+  int B, Hq, Hkv, group, max_pages, max_segs;
+  int has_pool;  // 0: no page pool, every output is an empty attention
 };
 
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hq) return;
-  const int b = gw / p.Hq;
-  int len = p.seq_lens[b];
-  const int cap = p.max_pages * kPage;
-  len = len < 0 ? 0 : (len > cap ? cap : len);
-  const int nsplit = ((len + kPage - 1) / kPage + kDecodePagesPerSplit - 1) / kDecodePagesPerSplit;
-  const float* base_o = p.ws_o + (size_t)gw * p.max_splits * kD;
-  const float* base_l = p.ws_lse + (size_t)gw * p.max_splits;
+  const int b = gw / p.Hq, h = gw % p.Hq;
+  const int npg = p.has_pool ? pages_of(p.seq_lens, p.max_pages, b) : 0;
+  int nseg = npg > 0 ? p.ws_nseg[b * p.Hkv + h / p.group] : 0;
+  nseg = nseg < 0 ? 0 : (nseg > p.max_segs ? p.max_segs : nseg);
+  const float* base_o = p.ws_o + (size_t)gw * p.max_segs * kD;
+  const float* base_l = p.ws_lse + (size_t)gw * p.max_segs;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float M = -INFINITY, L = 0.f;
-  // splits in groups of 32: lane s owns split s of the group
-  for (int s0 = 0; s0 < nsplit; s0 += 32) {
-    const int n = min(32, nsplit - s0);
+  // segments in groups of 32: lane s owns segment s of the group
+  for (int s0 = 0; s0 < nseg; s0 += 32) {
+    const int n = min(32, nseg - s0);
     const float l2 = lane < n ? base_l[s0 + lane] : -INFINITY;
     float gm = l2;
 #pragma unroll
@@ -410,13 +502,52 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   if (lane == 0 && p.lse) p.lse[gw] = (L > 0.f) ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// The pool [num_pages * 16 tokens, Hkv, D] bf16 as a 3-D tensor, box = one
+// page of one K/V head, 64 features (128 bytes, 128-byte swizzle).
+bool encode_pool(CUtensorMap* map, const void* pool, int num_pages, int Hkv) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)Hkv, (cuuint64_t)num_pages * kPage};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)Hkv * kD * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kPage};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// q [B * Hq rows, D] bf16, box = 32 rows x 64 features (128-byte swizzle).
+bool encode_q(CUtensorMap* map, const void* q, int rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kQRows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (a.D != kD || a.page_size != kPage) return -2;
   const int group = a.Hq / a.Hkv;
   if (group > 32) return -2;
-  const int max_splits = decode_max_splits(a.max_pages);
+  const int max_pages = a.max_pages > 0 ? a.max_pages : 1;
+  const int max_segs = decode_max_segments(max_pages);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -426,39 +557,53 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return fail_cuda("decode: cudaFuncSetAttribute", err);
     attr_set[dev] = true;
   }
-  SplitParams sp{};
-  sp.q = static_cast<const __nv_bfloat16*>(a.q);
-  sp.k_pages = static_cast<const __nv_bfloat16*>(a.k_pages);
-  sp.v_pages = static_cast<const __nv_bfloat16*>(a.v_pages);
-  sp.block_table = a.block_table;
-  sp.seq_lens = a.seq_lens;
-  sp.ws_o = static_cast<float*>(a.workspace);
-  sp.ws_lse = sp.ws_o + (size_t)a.B * a.Hq * max_splits * kD;
-  sp.B = a.B;
-  sp.Hq = a.Hq;
-  sp.Hkv = a.Hkv;
-  sp.group = group;
-  sp.num_pages = a.num_pages;
-  sp.max_pages = a.max_pages;
-  sp.max_splits = max_splits;
-  sp.scale_log2 = a.scale * kLog2e;
-  sp.bounds_check = (debug_flags() & 1) ? 1 : 0;
-  sp.status = device_status_word();
-  if (!sp.status) return fail_cuda("decode: status word", cudaGetLastError());
-  dim3 grid(max_splits, a.B * a.Hkv);
-  decode_split_kernel<<<grid, kThreads, kSmemBytes, stream>>>(sp);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return fail_cuda("decode: split launch", err);
+  float* ws_o = static_cast<float*>(a.workspace);
+  float* ws_lse = ws_o + (size_t)a.B * a.Hq * max_segs * kD;
+  int* ws_nseg = reinterpret_cast<int*>(ws_lse + (size_t)a.B * a.Hq * max_segs);
+  int* status = device_status_word();
+  if (!status) return fail_cuda("decode: status word", cudaGetLastError());
+  if (a.num_pages > 0 && a.max_pages > 0) {
+    SplitParams sp{};
+    sp.block_table = a.block_table;
+    sp.seq_lens = a.seq_lens;
+    sp.ws_o = ws_o;
+    sp.ws_lse = ws_lse;
+    sp.ws_nseg = ws_nseg;
+    sp.B = a.B;
+    sp.Hq = a.Hq;
+    sp.Hkv = a.Hkv;
+    sp.group = group;
+    sp.num_pages = a.num_pages;
+    sp.max_pages = a.max_pages;
+    sp.max_segs = max_segs;
+    sp.scale_log2 = a.scale * kLog2e;
+    sp.bounds_check = (debug_flags() & 1) ? 1 : 0;
+    sp.status = status;
+    sp.timeout_ns = wait_timeout_ns();
+    CUtensorMap tq, tk, tv;
+    if (!encode_q(&tq, a.q, a.B * a.Hq) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
+        !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv))
+      return fail_cuda("decode: tensor map", cudaErrorInvalidValue);
+    decode_split_kernel<<<kCtasPerSm * sm_count(), kThreads, kSmemBytes, stream>>>(tq, tk, tv, sp);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return fail_cuda("decode: split launch", err);
+  }
   CombineParams cp{};
-  cp.ws_o = sp.ws_o;
-  cp.ws_lse = sp.ws_lse;
+  cp.ws_o = ws_o;
+  cp.ws_lse = ws_lse;
+  cp.ws_nseg = ws_nseg;
   cp.seq_lens = a.seq_lens;
   cp.o = static_cast<__nv_bfloat16*>(a.o);
   cp.lse = a.lse;
   cp.B = a.B;
   cp.Hq = a.Hq;
-  cp.max_pages = a.max_pages;
-  cp.max_splits = max_splits;
+  cp.Hkv = a.Hkv;
+  cp.group = group;
+  cp.max_pages = max_pages;
+  cp.max_segs = max_segs;
+  // Without a pool the split kernel did not run and wrote no segment counts:
+  // the combine then treats every sequence as empty (O = 0, LSE = -inf).
+  cp.has_pool = (a.num_pages > 0 && a.max_pages > 0) ? 1 : 0;
   const int nw = a.B * a.Hq;
   decode_combine_kernel<<<(nw + 7) / 8, 256, 0, stream>>>(cp);
   err = cudaGetLastError();

@@ -50,13 +50,22 @@ int fail_cuda(const char* where, cudaError_t err);
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
-// Decode work split (shared by the workspace-size query and the launcher).
-#ifndef ATTN_DECODE_PAGES_PER_SPLIT
-#define ATTN_DECODE_PAGES_PER_SPLIT 32
+// Decode work partition.  Every CTA streams a contiguous share of all cached
+// pages of the batch, at least kDecodeMinChunk pages, so a sequence of P pages
+// is cut into at most ceil(P / kDecodeMinChunk) + 1 segments; each segment
+// leaves one partial (D floats + its log-sum-exp) per query head.
+#ifndef ATTN_DECODE_MIN_CHUNK
+#define ATTN_DECODE_MIN_CHUNK 32
 #endif
-constexpr int kDecodePagesPerSplit = ATTN_DECODE_PAGES_PER_SPLIT;  // 512 tokens per split CTA
-inline int decode_max_splits(int max_pages) {
-  return (max_pages + kDecodePagesPerSplit - 1) / kDecodePagesPerSplit;
+constexpr int kDecodeMinChunk = ATTN_DECODE_MIN_CHUNK;  // pages (512 tokens)
+inline int decode_max_segments(int max_pages) {
+  return (max_pages + kDecodeMinChunk - 1) / kDecodeMinChunk + 1;
+}
+// Workspace: partial outputs [B*Hq][S][D] f32, their LSE [B*Hq][S] f32 and the
+// segment count of every (sequence, K/V head) [B*Hq] int32, S = segments.
+inline size_t decode_workspace_bytes(int B, int Hq, int max_pages, int D) {
+  const size_t rows = (size_t)B * Hq, segs = (size_t)decode_max_segments(max_pages);
+  return rows * segs * (size_t)(D + 1) * 4 + rows * 4;
 }
 
 }  // namespace attn

@@ -123,8 +123,9 @@ ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
 
 /*
  * attn_decode_workspace_bytes -- size of the scratch buffer attn_decode_paged
- * needs for these sizes (split partials: per sequence, per split of 512
- * cached tokens, per query head, D + 1 floats).  Host only; never fails (0 for empty shapes).
+ * needs for these sizes: per query head of every sequence, up to
+ * ceil(max_pages_per_seq / 32) + 1 partial results of D + 1 floats, plus one
+ * int per (sequence, query head).  Host only; never fails (0 for empty shapes).
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D);
 

@@ -59,9 +59,10 @@ def test_status_strings_and_version(cdll):
 
 def test_workspace_size_formula(cdll):
     import attention_flash_attn_02_b200 as attn
-    # 512 tokens (32 pages of 16) per split; (D + 1) floats per (seq, head, split)
-    assert attn.attn_decode_workspace_bytes(64, 32, 512, 128) == 64 * 32 * 16 * 129 * 4
-    assert attn.attn_decode_workspace_bytes(2, 4, 33, 128) == 2 * 4 * 2 * 129 * 4
+    # a sequence of P pages is cut into at most ceil(P / 32) + 1 segments; each
+    # leaves D + 1 floats per query head; plus one int per (sequence, head)
+    assert attn.attn_decode_workspace_bytes(64, 32, 512, 128) == 64 * 32 * 17 * 129 * 4 + 64 * 32 * 4
+    assert attn.attn_decode_workspace_bytes(2, 4, 33, 128) == 2 * 4 * 3 * 129 * 4 + 2 * 4 * 4
     assert attn.attn_decode_workspace_bytes(0, 4, 33, 128) == 0
 
 
