@@ -63,6 +63,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_decode_workspace_bytes.restype = c_size_t
     lib.attn_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p, c_size_t, c_void_p]
     lib.attn_decode_paged.restype = c_int
+    lib.attn_decode_paged_noalloc.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p]
+    lib.attn_decode_paged_noalloc.restype = c_int
     lib.attn_last_device_error.argtypes = [c_void_p]
     lib.attn_last_device_error.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
@@ -175,6 +177,34 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: Optiona
                                float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _stream_handle(stream))
     _check(st, "attn_decode_paged")
+    return o, lse
+
+
+def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,
+                              o=None, lse=None, stream=None):
+    """attn_decode_paged without a workspace argument, for callers that cannot
+    allocate device memory when they run decode: the scratch is a fixed array
+    inside the library (ATTN_DECODE_NOALLOC_SCRATCH_BYTES).  Calls that overlap
+    on the GPU share that array and must not run concurrently.  Returns
+    (o bf16 [B,Hq,D], lse fp32 [B,Hq]); outputs may be passed in to avoid any
+    allocation in this wrapper too."""
+    import torch
+    lib = load()
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("attn_decode_paged_noalloc: block_table and seq_lens must be int32")
+    st = lib.attn_decode_paged_noalloc(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                                       _ptr(o), _ptr(lse), B, Hq, Hkv, D, page_size, num_pages, max_pages,
+                                       float(scale), _stream_handle(stream))
+    _check(st, "attn_decode_paged_noalloc")
     return o, lse
 
 

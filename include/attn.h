@@ -161,6 +161,36 @@ ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v
                                void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot
+ * allocate device memory at the call site (no counterpart in the pages this
+ * library follows).
+ *
+ * Who needs it: code running inside another runtime's execution hook (an
+ * engine plugin's enqueue, for instance) where that runtime owns all device
+ * memory and no allocation is allowed, or a service that must not grow its
+ * device footprint after start-up; a cudaMalloc there would also synchronise
+ * the device.  Here the decode scratch is a fixed device array compiled into
+ * the library (ATTN_DECODE_NOALLOC_SCRATCH_BYTES, held by every GPU that loads
+ * the library until the process exits), so the call allocates nothing:
+ * no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Arguments, layouts, supported sizes and results are those of
+ * attn_decode_paged, without the workspace.  Sizes whose scratch
+ * (attn_decode_workspace_bytes) exceeds the array return ATTN_ERR_INVALID
+ * before anything is launched, with the sizes in attn_last_error_message().
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the previous call's
+ * contents (nothing in it needs to start at zero); calls that overlap on the
+ * GPU -- different streams with no ordering between them -- race on it.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+ATTN_API int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                       const int* block_table, const int* seq_lens, void* o, float* lse,
+                                       int B, int Hq, int Hkv, int D, int page_size, int num_pages,
+                                       int max_pages_per_seq, float scale, attn_stream_t stream);
+
+/*
  * attn_last_device_error -- synchronises `stream`, then returns and clears the
  * status word the kernels write on the current device: ATTN_OK,
  * ATTN_ERR_TIMEOUT (a bounded wait inside a kernel ran out; the kernel
