@@ -31,6 +31,7 @@ ATTN_ERR_CUDA = -3
 ATTN_ERR_TIMEOUT = -4
 ATTN_ERR_BOUNDS = -5
 ATTN_DEBUG_BOUNDS = 1
+ATTN_DEBUG_STALL = 2
 
 _lib = None
 

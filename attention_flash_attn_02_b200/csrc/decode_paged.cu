@@ -66,6 +66,7 @@ struct SplitParams {
   int bounds_check;
   int* status;
   unsigned long long timeout_ns;
+  int stall;  // testing hook: the producer issues no loads, every wait runs out
 };
 
 struct DecSmem {
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       tma_prefetch_desc(&tm_v);
     }
     uint32_t n_st = 0, n_q = 0;
-    bool ok = true;
+    bool ok = !p.stall;
     Segments seg(p, lo, hi);
     while (seg.more() && ok) {
       int b, kvh, pg_lo, pg_hi, P;
@@ -580,6 +581,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sp.bounds_check = (debug_flags() & 1) ? 1 : 0;
     sp.status = status;
     sp.timeout_ns = wait_timeout_ns();
+    sp.stall = (debug_flags() & 2) ? 1 : 0;
     CUtensorMap tq, tk, tv;
     if (!encode_q(&tq, a.q, a.B * a.Hq) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
         !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv))

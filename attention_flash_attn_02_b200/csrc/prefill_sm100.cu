@@ -104,6 +104,7 @@ struct Params {
   float out_scale;   // 1 (bf16) or v_descale (fp8)
   int* status;
   unsigned long long timeout_ns;
+  int stall;  // testing hook: the producer issues no loads, every wait runs out
 };
 
 struct Unit {
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t seq = 0, nunit = 0;
-      bool ok = true;
+      bool ok = !p.stall;
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
         const Unit w = get_unit(u, p);
         if (w.nb <= 0) continue;
@@ -629,6 +630,7 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   p.status = device_status_word();
   if (!p.status) return fail_cuda("prefill: status word", cudaGetLastError());
   p.timeout_ns = wait_timeout_ns();
+  p.stall = (debug_flags() & 2) ? 1 : 0;
 
   CUtensorMap tq, tk, tv;
   const bool have_k = a.Lk > 0;

@@ -44,7 +44,7 @@ L2_FLUSH_BYTES = 256 << 20
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' side measurements")
@@ -97,58 +97,63 @@ def measured_peaks():
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi every 200 ms."""
+    """Samples SM clocks and throttle reasons of the GPU under test with
+    nvidia-smi every 200 ms from a background thread while the timed region
+    runs.  The device is matched by UUID, else by index, else it is the only
+    GPU nvidia-smi lists."""
 
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, uuid):
-        self.uuid = (uuid or "").lower()  # CUDA uuid of the device under test
-        self.proc = None
-        self.path = os.path.join("/tmp", f"attn_bench_clocks_{os.getpid()}.csv")
+    def __init__(self, uuid: str, index: int):
+        self.uuid = (uuid or "").lower().replace("gpu-", "").replace("-", "")
+        self.index = str(index)
+        self.rows = []
+        self._stop = None
+        self._thread = None
+
+    def _poll(self):
+        import threading  # noqa: F401
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits"],
+                                     capture_output=True, text=True, timeout=5).stdout
+                for line in out.splitlines():
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 10:
+                        self.rows.append(parts)
+            except Exception:
+                pass
+            self._stop.wait(0.2)
 
     def start(self):
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        import threading
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not sampled"], "samples": 0}
+        self._stop.set()
+        self._thread.join(timeout=10)
+        rows = self.rows
         norm = lambda u: u.lower().replace("gpu-", "").replace("-", "")  # noqa: E731
-        uuids = {norm(r[0]) for r in rows}
-        mine = [r for r in rows if self.uuid and norm(r[0]) == norm(self.uuid)]
-        seen = sorted(uuids)
-        rows = mine if mine else (rows if len(uuids) == 1 else [])
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["device not matched"],
-                    "samples": 0, "uuid": self.uuid, "seen": seen[:8]}
-        os.unlink(self.path)
-        if not rows:
+        mine = [r for r in rows if self.uuid and norm(r[1]) == self.uuid]
+        if not mine:
+            indices = {r[0] for r in rows}
+            mine = rows if len(indices) == 1 else [r for r in rows if r[0] == self.index]
+        if not mine:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "", 1).isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None  # noqa: E731
+        sm = [num(r[2]) for r in mine if num(r[2]) is not None]
+        mx = [num(r[3]) for r in mine if num(r[3]) is not None]
+        reasons = sorted({self.REASONS[i] for r in mine for i in range(4) if r[6 + i].lower() == "active"})
         load = [x for x in sm if x > 500] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(mine)}
 
 
 # ----------------------------------------------------------- CPU baseline
@@ -238,7 +243,7 @@ def run_ours(args):
         gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
         gpu_uuid = ""
-    clocks = ClockSampler(gpu_uuid)
+    clocks = ClockSampler(gpu_uuid, local)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()

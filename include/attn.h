@@ -206,11 +206,17 @@ ATTN_API const char* attn_status_str(int status);
  * attn_set_debug -- process-wide debug switches for later launches.
  *   flags bit 0 (ATTN_DEBUG_BOUNDS): decode checks every page id against
  *                num_pages and every token against seq_len.
+ *   flags bit 1 (ATTN_DEBUG_STALL): testing hook for failure detection --
+ *                the kernels' load producers issue nothing, so every bounded
+ *                wait runs out; the kernels release their resources, return,
+ *                and attn_last_device_error() reports ATTN_ERR_TIMEOUT.  The
+ *                outputs of such calls are undefined.
  *   wait_timeout_ns: limit of every bounded wait inside the kernels
  *                (0 = the default of 2 s).
  * Returns the previous flags.
  */
 #define ATTN_DEBUG_BOUNDS 1
+#define ATTN_DEBUG_STALL 2
 ATTN_API int attn_set_debug(int flags, unsigned long long wait_timeout_ns);
 
 /*
