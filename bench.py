@@ -38,6 +38,26 @@ METRIC = "attention fwd TFLOP/s (prefill) & decode HBM GB/s, % of B200 roofline"
 PREFILL = GQA_CAUSAL
 DECODE = MQA_DECODE
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# the ncu captures summarised under profiles/, valid only for the kernel
+# sources they were taken on (sha256 prefix of the files); a changed kernel
+# reports null until it is captured again.
+PROFILED_TRAFFIC = {
+    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "87167add744fa66f",
+                "bytes": 313_984_000 + 100_759_552, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
+    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "f4e47003e5793c86",
+               "bytes": 147_888_384 + 4_291_328, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
+}
+
+
+def profiled_traffic(kernel: str):
+    import hashlib
+    entry = PROFILED_TRAFFIC[kernel]
+    h = hashlib.sha256()
+    for f in entry["files"]:
+        with open(os.path.join(ROOT, "attention_flash_attn_02_b200", f), "rb") as fh:
+            h.update(fh.read())
+    return entry["bytes"] if h.hexdigest()[:16] == entry["sha"] else None
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -223,7 +243,7 @@ def run_ours(args):
         # than L2, then read another one so the written lines are flushed back
         # to HBM here rather than during the decode.
         flush.zero_()
-        flush_rd.sum()
+        flush_rd.view(torch.int32).sum(dtype=torch.int32)
         if ev is not None:
             ev[2].record(stream)
         attn.attn_decode_paged(dq, dkp, dvp, dbt, dsl, DECODE.scale, o=do, lse=dlse, workspace=ws)
@@ -349,14 +369,16 @@ def run_ours(args):
             "frac": round(achieved_pre / peak_t, 4),
             "frac_of_sustained": round(achieved_pre / peaks["bf16_tflops_sustained"], 4),
             "peak_source": f"{peak_src} bf16_tflops (burst)",
-            "traffic": None,
+            "traffic": profiled_traffic("prefill"),
+            "algorithmic_bytes": prefill_bytes(PREFILL),
         },
         "decode": {
             "value": round(dec_gbs, 1), "unit": "GB/s", "workload": DECODE.name,
             "us_per_call": round(dec_ms / K * 1e3, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved_dec, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(achieved_dec / peaks["hbm_gbs"], 4),
-                         "peak_source": f"{peak_src} hbm_gbs", "traffic": None},
+                         "peak_source": f"{peak_src} hbm_gbs", "traffic": profiled_traffic("decode"),
+                         "algorithmic_bytes": db},
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
