@@ -54,7 +54,7 @@ def up_to_date() -> bool:
 # setmaxnreg; the split assumes this launch register count (see
 # csrc/prefill_sm100.cu).  A different count could make the increase wait
 # forever, so the build refuses to produce such a library.
-PREFILL_LAUNCH_REGS = 168
+PREFILL_LAUNCH_REGS = 128
 
 
 def check_register_counts(ptxas_log: str) -> None:

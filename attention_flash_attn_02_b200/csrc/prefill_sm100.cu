@@ -43,17 +43,21 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per K/V block
-constexpr int kThreads = 384;  // 3 warpgroups
+constexpr int kThreads = 512;  // 4 warpgroups
 // Register split (setmaxnreg): the block launches with kLaunchRegs per thread
-// (384 threads x 168 fills the register file: 3 warps per SM sub-partition).
-// The producer/MMA warpgroup gives registers back and the two softmax
-// warpgroups take them.  The shares must add up to exactly the launch total
-// or the increase would wait forever: 2 * 200 + 104 = 3 * 168.  The build
-// checks with ptxas that the kernels launch with kLaunchRegs.
-constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 200;
-constexpr int kOtherRegs = 104;
-static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must match the launch total");
+// (512 threads x 128 fills the register file: 4 warps per SM sub-partition).
+// The producer/MMA warpgroup and the epilogue warpgroup give registers back and
+// the two softmax warpgroups take them.  Warps go round-robin to the four SM
+// sub-partitions, so each holds one warp of every warpgroup, and the shares
+// must add up to exactly its launch total or the increase would wait forever:
+// 2 * 192 + 88 + 40 = 4 * 128.
+// The build checks with ptxas that the kernels launch with kLaunchRegs.
+constexpr int kLaunchRegs = 128;
+constexpr int kSoftmaxRegs = 192;
+constexpr int kIssueRegs = 88;
+constexpr int kEpilogueRegs = 40;
+static_assert(2 * kSoftmaxRegs + kIssueRegs + kEpilogueRegs == 4 * kLaunchRegs,
+              "register split must match the launch total");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 // Of every 8 pairs of exponentials, this many are computed by the FMA-pipe
@@ -72,8 +76,8 @@ struct Cfg {
   static constexpr int BOX_BYTES = kBM * 128;            // one box: 128 rows x 128 B
   static constexpr int TILE_BYTES = kBM * ROW_BYTES;
 #ifndef ATTN_KV_STAGES_BIG
-#define ATTN_KV_STAGES_BIG 5
-#define ATTN_KV_STAGES_SMALL 12
+#define ATTN_KV_STAGES_BIG 4
+#define ATTN_KV_STAGES_SMALL 11
 #endif
   static constexpr int NS = TILE_BYTES >= 32768 ? ATTN_KV_STAGES_BIG : ATTN_KV_STAGES_SMALL;  // K/V ring stages
   static constexpr int MMA_K = FP8 ? 32 : 16;
@@ -84,7 +88,7 @@ struct Cfg {
   static constexpr uint32_t IDESC_PV = make_idesc(FP8 ? 0u : 1u, kBM, D, true);
   // shared memory: [Q0][Q1][stage 0..NS-1] (1024-aligned) + barriers
   static constexpr int SMEM_TILES = (2 + NS) * TILE_BYTES;
-  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align slack*/ + 512 /*barriers*/;
+  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align slack*/ + 4096 /*barriers, row statistics*/;
   static_assert(SMEM_BYTES <= 232448, "more than the 227 KB a CTA may use");
   static_assert(NBOX >= 1 && ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle rows");
   static_assert(TM_O1 + D <= 512, "TMEM budget");
@@ -113,6 +117,10 @@ struct Unit {
   int kvbh;   // b * Hkv + kv head
   int kb_lo;  // first K/V block
   int nb;     // number of K/V blocks (0: nothing visible)
+  // Per-tile fields by a runtime tile index, as selects (an indexed load
+  // would put the struct in local memory).
+  __device__ __forceinline__ int bh_of(int t) const { return t ? bh[1] : bh[0]; }
+  __device__ __forceinline__ int m0_of(int t) const { return t ? m0[1] : m0[0]; }
 };
 
 // Visible keys [lo, hi) of query row i (bottom-right causal alignment; window
@@ -191,11 +199,15 @@ struct Smem {
   uint64_t o_full[2], o_empty[2];
   uint64_t drain;
   uint64_t kv_full[12], kv_empty[12];
+  uint64_t st_full[2];        // row statistics of a unit written (128 arrivals)
   uint32_t tmem_base;
   int abort_flag;
+  float st_m[2][kBM];         // [tile][row] running max (log2 units) at unit end
+  float st_l[2][kBM];         // [tile][row] exact row sum
+  float st_r[2][kBM];         // [tile][row] sum of the rounded P
 };
 
-static_assert(sizeof(Smem) <= 512, "barrier block exceeds its reserve");
+static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserve");
 
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tiles_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* tiles_ptr = smem_raw + (tiles_addr - raw_addr);
   Smem& sm = *reinterpret_cast<Smem*>(tiles_ptr + C::SMEM_TILES);
-  const uint32_t q_addr[2] = {tiles_addr, tiles_addr + (uint32_t)C::TILE_BYTES};
+  auto q_addr = [&](int t) { return tiles_addr + (t ? (uint32_t)C::TILE_BYTES : 0u); };
   const uint32_t kv_addr0 = tiles_addr + 2u * C::TILE_BYTES;
 
   const int warp = threadIdx.x >> 5;
@@ -221,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[t], 128);
       mbar_init(&sm.o_full[t], 1);
       mbar_init(&sm.o_empty[t], 128);
+      mbar_init(&sm.st_full[t], 128);
     }
     mbar_init(&sm.drain, 1);
     for (int s = 0; s < C::NS; ++s) {
@@ -258,15 +271,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  if (warp >= 8) {
-    // Third warpgroup: hand registers back to the softmax warpgroups.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-  }
-  if (warp >= 10) {
+  // Each role branch sets its own register count first thing, so that no code
+  // is reachable under two different counts.
+  if (warp == 10 || warp == 11) {
     // spare warps of the third warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
+    finish();
+  } else if (warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kEpilogueRegs));
+    // ------------------------------------------------------------ epilogue
+    // One thread per query row of each tile: O = acc / sum (bf16) and
+    // LSE = (max + log2 sum) ln 2, off the softmax warps' critical path.
+    const int r = ((warp & 3) << 5) + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+    uint32_t nunit = 0;
+    bool ok = true;
+    for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
+      const Unit w = get_unit(u, p);
+      for (int t = 0; t < 2 && ok; ++t) {
+        const int row = w.m0_of(t) + r;
+        const bool row_valid = row < p.Lq;
+        float m = -INFINITY, l = 0.f, lr = 0.f;
+        if (w.nb > 0) {
+          ok = mbar_wait(&sm.st_full[t], nunit & 1, g) && mbar_wait(&sm.o_full[t], nunit & 1, g);
+          if (!ok) break;
+          tc_fence_after();
+          m = sm.st_m[t][r];
+          l = sm.st_l[t][r];
+          lr = sm.st_r[t][r];
+        }
+        const float inv = (lr > 0.f) ? p.out_scale / lr : 0.f;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)w.bh_of(t) * p.Lq + row) * D;
+        const uint32_t tO = tmem + (t == 0 ? C::TM_O0 : C::TM_O1) + lane_off;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t raw[16];
+          if (w.nb > 0) {
+            tmem_ld16(tO + c * 16, raw);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) raw[i] = 0u;
+          }
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(raw[2 * i]) * inv, __uint_as_float(raw[2 * i + 1]) * inv);
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+        if (row_valid && p.lse != nullptr)
+          p.lse[(size_t)w.bh_of(t) * p.Lq + row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+        if (w.nb > 0) {
+          tc_fence_before();
+          mbar_arrive(&sm.o_empty[t]);
+        }
+      }
+      if (w.nb > 0) ++nunit;
+    }
     finish();
   } else if (warp == 8) {
     // ------------------------------------------------------------ producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
     if (lane == 0) {
       uint32_t seq = 0, nunit = 0;
       bool ok = !p.stall;
@@ -279,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sm.q_full[t], C::TILE_BYTES);
 #pragma unroll
           for (int bx = 0; bx < C::NBOX; ++bx)
-            tma_load_3d(q_addr[t] + bx * C::BOX_BYTES, &tm_q, &sm.q_full[t], bx * C::BOX_ELEMS, w.m0[t], w.bh[t]);
+            tma_load_3d(q_addr(t) + bx * C::BOX_BYTES, &tm_q, &sm.q_full[t], bx * C::BOX_ELEMS, w.m0_of(t), w.bh_of(t));
         }
         for (int j = 0; j < w.nb && ok; ++j) {
           const int row = (w.kb_lo + j) * kBN;
@@ -311,33 +379,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     finish();
   } else if (warp == 9) {
     // ----------------------------------------------------------- MMA issue
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
     if (lane == 0) {
-      uint32_t seq = 0, nunit = 0, pcnt[2] = {0, 0};
+      // pcnt: K/V blocks whose P of both tiles has been consumed so far
+      uint32_t seq = 0, nunit = 0, pcnt = 0;
       bool ok = true;
-      const uint32_t tS[2] = {tmem + C::TM_S0, tmem + C::TM_S1};
-      const uint32_t tO[2] = {tmem + C::TM_O0, tmem + C::TM_O1};
+      auto tS = [&](int t) { return tmem + (t ? C::TM_S1 : C::TM_S0); };
+      auto tO = [&](int t) { return tmem + (t ? C::TM_O1 : C::TM_O0); };
+      // S_t = Q_t K^T: K-major operands; k-step kk starts kk*MMA_K elements
+      // into the 128-byte rows, boxes of 64 (bf16) columns are BOX_BYTES apart.
+      // Descriptors are built once per tile and advanced by adding
+      // (byte offset >> 4) to their start-address field (no carry: < 256 KB).
       auto issue_s = [&](int t, uint32_t k_stage_addr) {
+        const uint64_t a0 = sw128_desc(q_addr(t), 16, 1024);
+        const uint64_t b0 = sw128_desc(k_stage_addr, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
           const uint32_t byte_k = kk * C::MMA_K * C::EL;
-          const uint32_t off = (byte_k / 128) * C::BOX_BYTES + (byte_k % 128);
-          const uint64_t a = sw128_desc(q_addr[t] + off, 16, 1024);
-          const uint64_t b = sw128_desc(k_stage_addr + off, 16, 1024);
+          const uint32_t off = ((byte_k / 128) * C::BOX_BYTES + (byte_k % 128)) >> 4;
           if (FP8)
-            mma_f8_ss(tS[t], a, b, C::IDESC_S, kk > 0);
+            mma_f8_ss(tS(t), a0 + off, b0 + off, C::IDESC_S, kk > 0);
           else
-            mma_f16_ss(tS[t], a, b, C::IDESC_S, kk > 0);
+            mma_f16_ss(tS(t), a0 + off, b0 + off, C::IDESC_S, kk > 0);
         }
       };
+      // O_t (+)= P_t V: P from TMEM (over S_t), V MN-major, 128-byte column
+      // groups BOX_BYTES apart, k-step kk = MMA_K keys of 128-byte rows.
       auto issue_pv = [&](int t, uint32_t v_stage_addr, bool acc) {
+        const uint64_t b0 = sw128_desc(v_stage_addr, C::BOX_BYTES, 1024);
 #pragma unroll
         for (int kk = 0; kk < C::PV_KSTEPS; ++kk) {
-          const uint64_t b = sw128_desc(v_stage_addr + kk * C::MMA_K * 128, C::BOX_BYTES, 1024);
-          const uint32_t a = tS[t] + kk * (C::MMA_K * C::EL / 4);
+          const uint32_t a = tS(t) + kk * (C::MMA_K * C::EL / 4);
+          const uint32_t off = (kk * C::MMA_K * 128) >> 4;
           if (FP8)
-            mma_f8_ts(tO[t], a, b, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            mma_f8_ts(tO(t), a, b0 + off, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
           else
-            mma_f16_ts(tO[t], a, b, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            mma_f16_ts(tO(t), a, b0 + off, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
@@ -364,9 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool has_next = j + 1 < w.nb;
           const uint32_t skn = seq % C::NS;
           for (int t = 0; t < 2 && ok; ++t) {
-            ok = mbar_wait(&sm.p_full[t], pcnt[t] & 1, g);
+            ok = mbar_wait(&sm.p_full[t], pcnt & 1, g);
             if (!ok) break;
-            ++pcnt[t];
             if (j == 0 && nunit > 0) {
               ok = mbar_wait(&sm.o_empty[t], (nunit - 1) & 1, g);
               if (!ok) break;
@@ -385,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
+          ++pcnt;
           tc_commit(&sm.kv_empty[sv]);
           if (has_next) {
             tc_commit(&sm.kv_empty[skn]);
@@ -415,8 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
       const Unit w = get_unit(u, p);
-      const int row = w.m0[t] + r;
-      const bool row_valid = row < p.Lq;
+      const int row = w.m0_of(t) + r;
       // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
       // the MMA multiplies (normalises O so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
@@ -429,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++scnt;
           tc_fence_after();
           uint32_t sr[kBN];  // raw fp32 scores of this row
-          tmem_ld128(tS, sr);
+          tmem_ld64x2(tS, sr);
           const int key0 = (w.kb_lo + j) * kBN;
           if (!(lo <= key0 && key0 + kBN <= hi)) {  // diagonal / window-edge / ragged block
 #pragma unroll
@@ -525,37 +601,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&sm.p_full[t]);
         }
         if (!ok) break;
-        ok = mbar_wait(&sm.o_full[t], nunit & 1, g);
-        if (!ok) break;
-        tc_fence_after();
-      }
-      // Epilogue: O = acc / sum (bf16), LSE = (max + log2 sum) * ln 2.
-      const float inv_l = (l_rnd > 0.f) ? p.out_scale / l_rnd : 0.f;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)w.bh[t] * p.Lq + row) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t raw[32];
-        if (w.nb > 0) {
-          tmem_ld32(tO + c * 32, raw);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) raw[i] = 0u;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(raw[2 * i]) * inv_l, __uint_as_float(raw[2 * i + 1]) * inv_l);
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
-      }
-      if (row_valid && p.lse != nullptr)
-        p.lse[(size_t)w.bh[t] * p.Lq + row] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-      if (w.nb > 0) {
-        tc_fence_before();
-        mbar_arrive(&sm.o_empty[t]);
+        // hand the row statistics of this unit to the epilogue warpgroup
+        sm.st_m[t][r] = m_run;
+        sm.st_l[t][r] = l_run;
+        sm.st_r[t][r] = l_rnd;
+        mbar_arrive(&sm.st_full[t]);
         ++nunit;
       }
     }
