@@ -129,7 +129,7 @@ ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v
     return ATTN_ERR_INVALID;
   if (num_pages > 0 && (!k_pages || !v_pages || !aligned16(k_pages) || !aligned16(v_pages)))
     return ATTN_ERR_INVALID;
-  if (D != 128 || page_size != 16 || Hq / Hkv > 32) return ATTN_ERR_UNSUPPORTED;
+  if (D != 128 || page_size != 16 || Hq / Hkv > 128) return ATTN_ERR_UNSUPPORTED;
   const int mp = max_pages_per_seq > 0 ? max_pages_per_seq : 1;
   const size_t need = attn_decode_workspace_bytes(B, Hq, mp, D);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_INVALID;

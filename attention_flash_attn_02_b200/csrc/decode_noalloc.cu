@@ -18,7 +18,7 @@
 //     between them) race on it and give wrong results;
 //   * sizes whose scratch would exceed the array are rejected.
 // Nothing in the array has to start at zero: each call writes every partial
-// and every segment count it later reads, before reading it.
+// it later reads before reading it.
 #include <cstdio>
 #include <mutex>
 

@@ -4,26 +4,34 @@
 // per-sequence block table), for B200 (sm_100a).
 //
 // Two launches:
-//   decode_split_kernel   G = 3 CTAs per SM.  All cached pages of the batch,
+//   decode_split_kernel   2 CTAs per SM.  All cached pages of the batch,
 //       sequence after sequence (and K/V head after K/V head), form one list
 //       of T pages; CTA c streams the contiguous share [c T / G, (c+1) T / G)
 //       of it (at least kDecodeMinChunk pages), so every CTA moves the same
-//       number of bytes whatever the length mix.  Warp 2 is a TMA producer:
-//       it loads the 32 query rows of each sequence segment it meets and
-//       copies whole pages (K and V, 128-byte swizzled) straight from the pool
-//       into a 6-stage ring tracked by mbarriers.  Warps 0 and 1 take query
-//       rows [0, 16) and [16, 32) of the K/V group and compute S = q K^T and
-//       O += P V on the tensor cores (mma.sync m16n8k16 bf16 -> fp32) with the
-//       online-softmax recurrence; at the end of a segment they write one
-//       partial (normalised o, log2-sum-exp) per query head.
+//       number of bytes whatever the length mix.  Per CTA:
+//         warp 4       TMA producer: the query rows of each (sequence, K/V
+//                      head) segment it meets, and blocks of pages (K and V,
+//                      128-byte swizzled) gathered straight from the pool into
+//                      a ring; page ids come from the block table.
+//         warp 5       allocates TMEM; one thread issues the tensor-core work
+//                      of each block: S = Q K^T (tcgen05, M = 128 query rows
+//                      of which the K/V group's heads are the first `group`,
+//                      N = 16 per loaded page) into one of two TMEM S
+//                      buffers, then O += P V (P read back from TMEM over S).
+//         warps 0..3   softmax, one thread per query head (TMEM lane): online
+//                      softmax over each block's scores, P written back to
+//                      TMEM as bf16; at the end of a segment the normalised
+//                      partial o and its log2-sum-exp go to the workspace.
+//                      Only ceil(group / 32) of them have rows.
 //   decode_combine_kernel one warp per (sequence, query head) merges the
 //       partials: M = max_s lse_s, O = sum_s 2^(lse_s - M) o_s / sum_s
-//       2^(lse_s - M), LSE = (M + log2 sum) ln 2.  This is the rescaling step of
-//       the online softmax (page "003-注意力机制详解...", §二) applied once
-//       across segments.
+//       2^(lse_s - M), LSE = (M + log2 sum) ln 2 -- the rescaling step of the
+//       online softmax (page "003-注意力机制详解...", §二) taken once across
+//       segments.  It is launched as a programmatic dependent of the split
+//       kernel and finds each pair's segments from seq_lens itself, so after
+//       the split kernel ends it needs one round of loads.
 // All query heads of a K/V group share every gathered page (MQA/GQA: the
-// tqpw.cn article §2.1/§3.1), which is what makes the tensor cores necessary:
-// with 32 heads per K/V head, a SIMT dot product would be compute-bound.
+// tqpw.cn article §2.1/§3.1): one MMA serves the whole group.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <cstdint>
@@ -36,32 +44,34 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kPage = 16;
-constexpr int kThreads = 96;                 // 2 consumer warps + 1 producer warp
-#ifndef ATTN_DECODE_STAGES
-#define ATTN_DECODE_STAGES 6
-#define ATTN_DECODE_CTAS_PER_SM 3
-#endif
-constexpr int kStages = ATTN_DECODE_STAGES;
-constexpr int kCtasPerSm = ATTN_DECODE_CTAS_PER_SM;
-constexpr int kHalfBox = kPage * 128;        // 16 tokens x 64 features (bf16): 2 KB
-constexpr int kPageBytes = 2 * kHalfBox;     // K (or V) of one page: 4 KB
-constexpr int kStageBytes = 2 * kPageBytes;  // K and V of one page: 8 KB
-constexpr int kQRows = 32;                   // query rows per K/V group tile
-constexpr int kQBox = kQRows * 128;          // 32 rows x 64 features: 4 KB
-constexpr int kQBytes = 2 * kQBox;           // 8 KB per query slot
-constexpr int kRingOff = 2 * kQBytes;        // two query slots, then the ring
-constexpr int kSmemBytes = 1024 + kRingOff + kStages * kStageBytes + 256;
+// Blocks of 4 pages (64 tokens) in a 3-stage ring of 96 KB, two CTAs per SM
+// with 256 TMEM columns each.  (Measured on B200 against 2-page blocks with
+// two CTAs per SM and 8-page blocks with one: 4 pages was fastest.)
+constexpr int kBlkPages = 4;                    // pages per block
+constexpr int kBlkTok = kBlkPages * kPage;      // 64 tokens per block
+constexpr int kHalf = kBlkTok * 128;            // a block's 64-feature half (bf16): 8 KB
+constexpr int kPageHalf = kPage * 128;          // one page's 64-feature half: 2 KB
+constexpr int kStageBytes = 4 * kHalf;          // K half 0, K half 1, V half 0, V half 1
+constexpr int kCtasPerSm = 2;
+constexpr int kStages = 3;
+constexpr int kThreads = 192;                   // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr int kMaxGroup = 128;                  // query heads per K/V head
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmS0 = 0, kTmS1 = kBlkTok, kTmO = 2 * kBlkTok;
+static_assert(kTmO + kD <= kTmemCols, "TMEM budget");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kIdescPV = make_idesc(1u, 128, kD, true);
 
 struct SplitParams {
   const int* block_table;
   const int* seq_lens;
   float* ws_o;    // [B * Hq][S][kD] normalised partial outputs
   float* ws_lse;  // [B * Hq][S] log2-sum-exp of each partial
-  int* ws_nseg;   // [B * Hkv] segments of each (sequence, K/V head)
   int B, Hq, Hkv, group, num_pages, max_pages, max_segs;
+  int q_half;      // bytes of one 64-feature half of a query tile
+  int sm_warps;    // softmax warps with rows: ceil(group / 32)
   float scale_log2;
   int bounds_check;
   int* status;
@@ -70,13 +80,22 @@ struct SplitParams {
 };
 
 struct DecSmem {
-  uint64_t full[kStages], empty[kStages];
-  uint64_t qfull[2], qempty[2];
-  int valid[kStages];
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t pv_done, o_full, o_empty, drain;
+  uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(DecSmem) <= 256, "barrier block exceeds its reserve");
-static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "CTAs per SM do not fit in shared memory");
+constexpr int kBarBytes = 256;
+static_assert(sizeof(DecSmem) <= kBarBytes, "barrier block exceeds its reserve");
+// Shared memory: [query slot 0][query slot 1][ring][barriers], the base
+// 1024-byte aligned.  Two CTAs must fit on an SM (233472 bytes, 1 KB of it
+// reserved per CTA) and a third must not (TMEM holds two CTAs' columns).
+__host__ __device__ constexpr int dec_smem_bytes(int q_half) { return 4 * q_half + kStages * kStageBytes + kBarBytes; }
+static_assert(kCtasPerSm * (dec_smem_bytes(32 * 128) + 1024) <= 233472, "the CTAs of an SM must fit");
+static_assert((kCtasPerSm + 1) * (dec_smem_bytes(8 * 128) + 1024) > 233472, "one CTA more must not fit");
+static_assert(dec_smem_bytes(kMaxGroup * 128) <= 232448, "a CTA may use at most 227 KB");
 
 __device__ __forceinline__ int len_of(const int* seq_lens, int max_pages, int b) {
   const int n = seq_lens[b], cap = max_pages * kPage;
@@ -97,20 +116,32 @@ struct Segments {
   long long x;    // next page of the list
   long long pre;  // list index of the first page of the current (b, kvh)
   int b, kvh, P;  // current sequence, K/V head, its page count
-  __device__ Segments(const SplitParams& p_, long long lo, long long hi_) : p(p_), hi(hi_), x(lo) {
+  // Called by all 32 lanes of a warp: finds the sequence holding list page
+  // `lo` with a warp-wide inclusive scan of the sequences' page counts, 32
+  // sequences per step (lo < T, so some sequence holds it).
+  __device__ Segments(const SplitParams& p_, long long lo, long long hi_, int lane)
+      : p(p_), hi(hi_), x(lo), pre(0), b(0), kvh(0), P(0) {
     long long c = 0;
-    b = 0;
-    kvh = 0;
-    P = 0;
-    pre = 0;
-    for (; b < p.B; ++b) {
-      P = pages_of(p.seq_lens, p.max_pages, b);
-      if (lo < c + (long long)p.Hkv * P) {
-        kvh = (int)((lo - c) / P);
-        pre = c + (long long)kvh * P;
+    for (int b0 = 0; b0 < p.B; b0 += 32) {
+      const int bl = b0 + lane;
+      const long long w = bl < p.B ? (long long)p.Hkv * pages_of(p.seq_lens, p.max_pages, bl) : 0;
+      long long inc = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, c + inc > lo);
+      if (hit) {
+        const int L = __ffs(hit) - 1;  // first sequence whose pages reach past lo
+        const long long excl = c + __shfl_sync(0xffffffffu, inc - w, L);
+        b = b0 + L;
+        P = pages_of(p.seq_lens, p.max_pages, b);
+        kvh = (int)((lo - excl) / P);
+        pre = excl + (long long)kvh * P;
         return;
       }
-      c += (long long)p.Hkv * P;
+      c += __shfl_sync(0xffffffffu, inc, 31);
     }
   }
   __device__ bool more() const { return x < hi; }
@@ -135,323 +166,74 @@ struct Segments {
   }
 };
 
-// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled
-// TMA box (rows of 128 bytes, base 1024-aligned).
-__device__ __forceinline__ uint32_t sw128(int r, int c) {
-  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  // Total pages T of the batch and this CTA's share.
-  long long T = 0;
-  for (int b = 0; b < p.B; ++b) T += (long long)p.Hkv * pages_of(p.seq_lens, p.max_pages, b);
+// Number of CTAs of the split grid that own pages, for T pages in all.
+__device__ __forceinline__ long long split_ctas(long long T, int grid) {
   long long G = T / kDecodeMinChunk;
-  if (G > (long long)gridDim.x) G = gridDim.x;
-  if (G < 1) G = 1;
-  const int c = blockIdx.x;
-  if (T == 0 || c >= G) return;
-  const long long lo = c * T / G, hi = (c + 1) * T / G;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t s_q = base;                // 2 query slots of 8 KB
-  const uint32_t s_ring = base + kRingOff;  // kStages x 8 KB
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(base_ptr + kRingOff + kStages * kStageBytes);
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 2);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.qfull[s], 1);
-      mbar_init(&sm.qempty[s], 2);
-    }
-    sm.abort_flag = 0;
-    fence_mbarrier_init();
-  }
-  __syncthreads();
-  const WaitGuard g{&sm.abort_flag, p.status, p.timeout_ns, true};
-  const WaitGuard g_drain{&sm.abort_flag, p.status, p.timeout_ns, false};
-
-  if (warp == 2) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-    }
-    uint32_t n_st = 0, n_q = 0;
-    bool ok = !p.stall;
-    Segments seg(p, lo, hi);
-    while (seg.more() && ok) {
-      int b, kvh, pg_lo, pg_hi, P;
-      long long pre;
-      seg.take(b, kvh, pg_lo, pg_hi, pre, P);
-      if (lane == 0) {  // query rows of this (sequence, K/V head)
-        const uint32_t qs = n_q & 1;
-        if (n_q >= 2) ok = mbar_wait(&sm.qempty[qs], ((n_q >> 1) - 1) & 1, g);
-        if (ok) {
-          mbar_arrive_expect_tx(&sm.qfull[qs], kQBytes);
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(s_q + qs * kQBytes + h * kQBox, &tm_q, &sm.qfull[qs], h * 64, b * p.Hq + kvh * p.group);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++n_q;
-      for (int k0 = pg_lo; k0 < pg_hi && ok; k0 += 32) {
-        // 32 page ids at a time, one per lane
-        int id = -1;
-        if (k0 + lane < pg_hi) {
-          id = p.block_table[(size_t)b * p.max_pages + k0 + lane];
-          if (p.bounds_check && (id < 0 || id >= p.num_pages)) {
-            atomicExch(p.status, kErrBounds);
-            id = -1;
-          }
-        }
-        const int kn = pg_hi - k0 < 32 ? pg_hi - k0 : 32;
-        for (int k = 0; k < kn && ok; ++k) {
-          const int pid = __shfl_sync(0xffffffffu, id, k);
-          if (lane == 0) {
-            const uint32_t st = n_st % kStages;
-            if (n_st >= (uint32_t)kStages) ok = mbar_wait(&sm.empty[st], ((n_st / kStages) - 1) & 1, g);
-            if (ok) {
-              sm.valid[st] = pid >= 0;
-              mbar_arrive_expect_tx(&sm.full[st], pid >= 0 ? kStageBytes : 0);
-              if (pid >= 0) {
-                const uint32_t dst = s_ring + st * kStageBytes;
-                for (int h = 0; h < 2; ++h) {
-                  tma_load_3d(dst + h * kHalfBox, &tm_k, &sm.full[st], h * 64, kvh, pid * kPage);
-                  tma_load_3d(dst + kPageBytes + h * kHalfBox, &tm_v, &sm.full[st], h * 64, kvh, pid * kPage);
-                }
-              }
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          ++n_st;
-        }
-      }
-    }
-    if (lane == 0) {
-      // Drain: the last loads of every slot have landed before the CTA exits.
-      for (uint32_t s = (n_st > (uint32_t)kStages ? n_st - kStages : 0); s < n_st; ++s)
-        mbar_wait(&sm.full[s % kStages], (s / kStages) & 1, g_drain);
-      for (uint32_t s = (n_q > 2u ? n_q - 2 : 0); s < n_q; ++s) mbar_wait(&sm.qfull[s & 1], (s >> 1) & 1, g_drain);
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  const int mt = warp;  // query rows [16 mt, 16 mt + 16) of the group
-  const int mi = lane >> 3, rr = lane & 7;
-  const float sl2 = p.scale_log2;
-  uint32_t n_st = 0, n_q = 0;
-  bool ok = true;
-  Segments seg(p, lo, hi);
-  while (seg.more() && ok) {
-    int b, kvh, pg_lo, pg_hi, P;
-    long long pre;
-    seg.take(b, kvh, pg_lo, pg_hi, pre, P);
-    const int len = len_of(p.seq_lens, p.max_pages, b);
-    const uint32_t qs = n_q & 1;
-    ok = mbar_wait(&sm.qfull[qs], (n_q >> 1) & 1, g);
-    if (!ok) break;
-    ++n_q;
-    uint32_t qa[kD / 16][4];
-#pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk)
-      ldsm_x4(s_q + qs * kQBytes + (kk >> 2) * kQBox + sw128(mt * 16 + (mi & 1) * 8 + rr, (kk & 3) * 2 + (mi >> 1)),
-              qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.qempty[qs]);  // query fragments are in registers
-
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY};
-    // per-lane partial row sums: exact fp32 (for the LSE) and of the rounded
-    // P the tensor cores multiply (normalises o)
-    float l_part[2] = {0.f, 0.f}, r_part[2] = {0.f, 0.f};
-
-    for (int k = pg_lo; k < pg_hi; ++k) {
-      const uint32_t st = n_st % kStages;
-      ok = mbar_wait(&sm.full[st], (n_st / kStages) & 1, g);
-      if (!ok) break;
-      ++n_st;
-      if (sm.valid[st]) {
-        const uint32_t sk = s_ring + st * kStageBytes;
-        const uint32_t sv = sk + kPageBytes;
-        // S = q K^T for 16 query rows x 16 tokens; even and odd k-steps in
-        // separate accumulators (two independent MMA chains)
-        float s[2][4], s2[2][4];
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] = s2[n][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(sk + (kk >> 2) * kHalfBox + sw128((mi >> 1) * 8 + rr, (kk & 3) * 2 + (mi & 1)), b0, b1, b2, b3);
-          if (kk & 1) {
-            mma_bf16(s2[0], qa[kk], b0, b1);
-            mma_bf16(s2[1], qa[kk], b2, b3);
-          } else {
-            mma_bf16(s[0], qa[kk], b0, b1);
-            mma_bf16(s[1], qa[kk], b2, b3);
-          }
-        }
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
-        // mask tokens past the end of the sequence
-        const int base_tok = k * kPage + (lane & 3) * 2;
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int tok = base_tok + n * 8 + (e & 1);
-            s[n][e] = tok < len ? s[n][e] * sl2 : -INFINITY;
-          }
-        // online softmax for rows r (e = 0,1) and r + 8 (e = 2,3)
-        float alpha[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float mx = fmaxf(fmaxf(s[0][2 * h], s[0][2 * h + 1]), fmaxf(s[1][2 * h], s[1][2 * h + 1]));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          alpha[h] = 1.f;
-          if (mx > m_run[h] + kRescaleThreshold) {
-            alpha[h] = ex2_approx(m_run[h] - mx);
-            m_run[h] = mx;
-          }
-          l_part[h] *= alpha[h];
-          r_part[h] *= alpha[h];
-        }
-        if (alpha[0] != 1.f || alpha[1] != 1.f) {
-#pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            o[n][0] *= alpha[0];
-            o[n][1] *= alpha[0];
-            o[n][2] *= alpha[1];
-            o[n][3] *= alpha[1];
-          }
-        }
-        uint32_t pa[4];
-        {
-          const float nm0 = m_run[0] == -INFINITY ? 0.f : -m_run[0];
-          const float nm1 = m_run[1] == -INFINITY ? 0.f : -m_run[1];
-          float pv[2][4];
-#pragma unroll
-          for (int n = 0; n < 2; ++n) {
-            pv[n][0] = ex2_approx(s[n][0] + nm0);
-            pv[n][1] = ex2_approx(s[n][1] + nm0);
-            pv[n][2] = ex2_approx(s[n][2] + nm1);
-            pv[n][3] = ex2_approx(s[n][3] + nm1);
-            l_part[0] += pv[n][0] + pv[n][1];
-            l_part[1] += pv[n][2] + pv[n][3];
-          }
-          pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
-          pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
-          pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
-          pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
-          r_part[0] += sum_bf16x2(pa[0]) + sum_bf16x2(pa[2]);
-          r_part[1] += sum_bf16x2(pa[1]) + sum_bf16x2(pa[3]);
-        }
-        // O += P V over 16 tokens x 128 features
-#pragma unroll
-        for (int n = 0; n < 16; n += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sv + (n >> 3) * kHalfBox + sw128((mi & 1) * 8 + rr, (n & 7) + (mi >> 1)), b0, b1, b2, b3);
-          mma_bf16(o[n], pa, b0, b1);
-          mma_bf16(o[n + 1], pa, b2, b3);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[st]);
-    }
-    if (!ok) break;
-    // One partial per query row of this warp for this segment.
-    const int sidx = c - owner(pre, T, (int)G);
-    if (sidx < 0 || sidx >= p.max_segs) {  // cannot happen with chunks >= kDecodeMinChunk pages
-      if (lane == 0) atomicExch(p.status, kErrBounds);
-      continue;
-    }
-    const int r0 = lane >> 2;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float l = l_part[h], lr = r_part[h];
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      lr += __shfl_xor_sync(0xffffffffu, lr, 1);
-      lr += __shfl_xor_sync(0xffffffffu, lr, 2);
-      const int row = mt * 16 + r0 + 8 * h;
-      if (row < p.group) {
-        const size_t rec = ((size_t)b * p.Hq + kvh * p.group + row) * p.max_segs + sidx;
-        const float inv = lr > 0.f ? 1.f / lr : 0.f;
-        float* dst = p.ws_o + rec * kD + (lane & 3) * 2;
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-          *reinterpret_cast<float2*>(dst + n * 8) = make_float2(o[n][2 * h] * inv, o[n][2 * h + 1] * inv);
-        if ((lane & 3) == 0) p.ws_lse[rec] = l > 0.f ? m_run[h] + __log2f(l) : -INFINITY;
-      }
-    }
-    if (sidx == 0 && mt == 0 && lane == 0)
-      p.ws_nseg[b * p.Hkv + kvh] = owner(pre + P - 1, T, (int)G) - owner(pre, T, (int)G) + 1;
-  }
+  if (G > (long long)grid) G = grid;
+  return G < 1 ? 1 : G;
 }
 
 struct CombineParams {
   const float* ws_o;
   const float* ws_lse;
-  const int* ws_nseg;
   const int* seq_lens;
   __nv_bfloat16* o;
   float* lse;
   int B, Hq, Hkv, group, max_pages, max_segs;
-  int has_pool;  // 0: no page pool, every output is an empty attention
+  int split_grid;  // CTAs launched for the split kernel
+  int has_pool;    // 0: no page pool, every output is an empty attention
 };
 
+// One warp per (sequence, query head).  Before waiting for the split kernel
+// it works out, from seq_lens alone, which CTAs hold that pair's segments
+// (the same partition the split kernel used); after the wait, lane s reads
+// segment s's log2-sum-exp while every lane reads its 4 features of up to 8
+// partials at once.
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (gw >= p.B * p.Hq) return;
-  const int b = gw / p.Hq, h = gw % p.Hq;
-  const int npg = p.has_pool ? pages_of(p.seq_lens, p.max_pages, b) : 0;
-  int nseg = npg > 0 ? p.ws_nseg[b * p.Hkv + h / p.group] : 0;
-  nseg = nseg < 0 ? 0 : (nseg > p.max_segs ? p.max_segs : nseg);
-  const float* base_o = p.ws_o + (size_t)gw * p.max_segs * kD;
+  if (gw >= p.B * p.Hq) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }
+  const int b = gw / p.Hq, h = gw % p.Hq, kvh = h / p.group;
+  int nseg = 0;
+  if (p.has_pool) {
+    // pages of sequences before b, and in all (seq_lens is an input of the
+    // split kernel, complete before it started)
+    long long before = 0, T = 0;
+    for (int bb = lane; bb < p.B; bb += 32) {
+      const long long w = pages_of(p.seq_lens, p.max_pages, bb);
+      T += w;
+      if (bb < b) before += w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      T += __shfl_xor_sync(0xffffffffu, T, o);
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+    }
+    T *= p.Hkv;
+    const int P = pages_of(p.seq_lens, p.max_pages, b);
+    if (P > 0 && T > 0) {
+      const long long G = split_ctas(T, p.split_grid);
+      const long long pre = before * p.Hkv + (long long)kvh * P;
+      nseg = owner(pre + P - 1, T, (int)G) - owner(pre, T, (int)G) + 1;
+      nseg = nseg > p.max_segs ? p.max_segs : nseg;
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the split kernel's partials are complete
+  const float* base_o = p.ws_o + (size_t)gw * p.max_segs * kD + lane * 4;
   const float* base_l = p.ws_lse + (size_t)gw * p.max_segs;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float M = -INFINITY, L = 0.f;
-  // segments in groups of 32: lane s owns segment s of the group
   for (int s0 = 0; s0 < nseg; s0 += 32) {
-    const int n = min(32, nseg - s0);
-    const float l2 = lane < n ? base_l[s0 + lane] : -INFINITY;
+    const int n = nseg - s0 < 32 ? nseg - s0 : 32;
+    const float l2 = lane < n ? __ldcg(base_l + s0 + lane) : -INFINITY;
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = u < n ? __ldcg(reinterpret_cast<const float4*>(base_o + (size_t)(s0 + u) * kD))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
     float gm = l2;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
@@ -469,30 +251,23 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
     L += ws;
-    int s = 0;
-    for (; s + 4 <= n; s += 4) {  // four independent loads in flight
-      float4 v[4];
-      float wv[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        v[u] = *reinterpret_cast<const float4*>(base_o + (size_t)(s0 + s + u) * kD + lane * 4);
-        wv[u] = __shfl_sync(0xffffffffu, w, s + u);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc.x += wv[u] * v[u].x;
-        acc.y += wv[u] * v[u].y;
-        acc.z += wv[u] * v[u].z;
-        acc.w += wv[u] * v[u].w;
+    for (int u = 0; u < 8; ++u) {
+      const float wv = __shfl_sync(0xffffffffu, w, u);
+      if (u < n) {
+        acc.x += wv * v[u].x;
+        acc.y += wv * v[u].y;
+        acc.z += wv * v[u].z;
+        acc.w += wv * v[u].w;
       }
     }
-    for (; s < n; ++s) {
-      const float4 v = *reinterpret_cast<const float4*>(base_o + (size_t)(s0 + s) * kD + lane * 4);
-      const float wv = __shfl_sync(0xffffffffu, w, s);
-      acc.x += wv * v.x;
-      acc.y += wv * v.y;
-      acc.z += wv * v.z;
-      acc.w += wv * v.w;
+    for (int u = 8; u < n; ++u) {  // more than 8 segments in this group of 32
+      const float4 vv = __ldcg(reinterpret_cast<const float4*>(base_o + (size_t)(s0 + u) * kD));
+      const float wv = __shfl_sync(0xffffffffu, w, u);
+      acc.x += wv * vv.x;
+      acc.y += wv * vv.y;
+      acc.z += wv * vv.z;
+      acc.w += wv * vv.w;
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -502,6 +277,388 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   *reinterpret_cast<uint2*>(p.o + (size_t)gw * kD + lane * 4) = packed;
   if (lane == 0 && p.lse) p.lse[gw] = (L > 0.f) ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  {
+    // Pull this CTA's slice of the block table toward L2 now; the page ids it
+    // will read are only known once the page counts below are summed.
+    const size_t tbytes = (size_t)p.B * p.max_pages * 4;
+    const size_t per = ((tbytes + gridDim.x - 1) / gridDim.x + 127) / 128 * 128;
+    const size_t off = (size_t)blockIdx.x * per + (size_t)tid * 128;
+    if (tid * 128 < per && off < tbytes)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(p.block_table) + off));
+  }
+  // Total pages T of the batch and this CTA's share.  Every warp sums the
+  // page counts itself, lane l taking sequences l, l + 32, ... (independent
+  // loads, then a shuffle reduction), so no warp waits for another.
+  long long T = 0;
+  for (int b = lane; b < p.B; b += 32) T += pages_of(p.seq_lens, p.max_pages, b);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
+  T *= p.Hkv;
+  const long long G = split_ctas(T, gridDim.x);
+  const int c = blockIdx.x;
+  // The combine launch may start now: it waits for this grid's completion
+  // (griddepcontrol.wait) before it reads any partial.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (T == 0 || c >= G) return;
+  const long long lo = c * T / G, hi = (c + 1) * T / G;
+
+  const uint32_t base = smem_u32(smem_raw);
+  if (base & 1023u) {  // the layout below needs a 1024-byte aligned base
+    if (tid == 0) atomicExch(p.status, kErrBounds);
+    return;
+  }
+  const uint32_t q_slot = 2u * p.q_half;
+  const uint32_t s_q = base;                       // two query slots
+  const uint32_t s_ring = base + 2u * q_slot;      // kStages x 32 KB
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw + 2u * q_slot + kStages * kStageBytes);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.q_full[s], 1);
+      mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], p.sm_warps);
+    }
+    mbar_init(&sm.pv_done, 1);
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.o_empty, p.sm_warps);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitGuard g{&sm.abort_flag, p.status, p.timeout_ns, true};
+  const WaitGuard g_drain{&sm.abort_flag, p.status, p.timeout_ns, false};
+  // Teardown at the end of every role: all threads meet, then the owner warp
+  // releases TMEM.
+  auto finish = [&]() {
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+    if (warp == 5) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    uint32_t n_blk = 0, n_q = 0;
+    bool ok = !p.stall;
+    Segments seg(p, lo, hi, lane);
+    while (seg.more() && ok) {
+      int b, kvh, pg_lo, pg_hi, P;
+      long long pre;
+      seg.take(b, kvh, pg_lo, pg_hi, pre, P);
+      if (lane == 0) {  // the K/V group's query rows
+        const uint32_t qs = n_q & 1;
+        if (n_q >= 2) ok = mbar_wait(&sm.q_empty[qs], ((n_q >> 1) - 1) & 1, g);
+        if (ok) {
+          mbar_arrive_expect_tx(&sm.q_full[qs], 2u * p.group * 128u);
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(s_q + qs * q_slot + h * p.q_half, &tm_q, &sm.q_full[qs], h * 64,
+                        b * p.Hq + kvh * p.group);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++n_q;
+      for (int k0 = pg_lo; k0 < pg_hi && ok; k0 += 32) {
+        // 32 page ids at a time, one per lane (32 is a whole number of blocks)
+        int id = 0;
+        if (k0 + lane < pg_hi) {
+          id = p.block_table[(size_t)b * p.max_pages + k0 + lane];
+          if (p.bounds_check && (id < 0 || id >= p.num_pages)) {
+            atomicExch(p.status, kErrBounds);
+            id = p.num_pages;  // past the pool: the copy reads zeros
+          }
+        }
+        const int kn = pg_hi - k0 < 32 ? pg_hi - k0 : 32;
+        for (int kb = 0; kb < kn && ok; kb += kBlkPages) {
+          const int nv = kn - kb < kBlkPages ? kn - kb : kBlkPages;
+          int pid[kBlkPages];
+#pragma unroll
+          for (int i = 0; i < kBlkPages; ++i) pid[i] = __shfl_sync(0xffffffffu, id, (kb + i) & 31);
+          if (lane == 0) {
+            const uint32_t st = n_blk % kStages;
+            if (n_blk >= (uint32_t)kStages) ok = mbar_wait(&sm.kv_empty[st], ((n_blk / kStages) - 1) & 1, g);
+            if (ok) {
+              mbar_arrive_expect_tx(&sm.kv_full[st], (uint32_t)nv * 4u * kPageHalf);
+              const uint32_t dst = s_ring + st * kStageBytes;
+              for (int i = 0; i < nv; ++i) {
+                const int tok = pid[i] * kPage;
+                const uint32_t d = dst + i * kPageHalf;
+                tma_load_3d(d, &tm_k, &sm.kv_full[st], 0, kvh, tok);
+                tma_load_3d(d + kHalf, &tm_k, &sm.kv_full[st], 64, kvh, tok);
+                tma_load_3d(d + 2 * kHalf, &tm_v, &sm.kv_full[st], 0, kvh, tok);
+                tma_load_3d(d + 3 * kHalf, &tm_v, &sm.kv_full[st], 64, kvh, tok);
+              }
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++n_blk;
+        }
+      }
+    }
+    if (lane == 0) {
+      // Drain: the last loads of every slot have landed before the CTA exits.
+      for (uint32_t s = (n_blk > (uint32_t)kStages ? n_blk - kStages : 0); s < n_blk; ++s)
+        mbar_wait(&sm.kv_full[s % kStages], (s / kStages) & 1, g_drain);
+      for (uint32_t s = (n_q > 2u ? n_q - 2 : 0); s < n_q; ++s) mbar_wait(&sm.q_full[s & 1], (s >> 1) & 1, g_drain);
+    }
+    finish();
+  } else if (warp == 5) {
+    // ----------------------------------------------------------- MMA issue
+    Segments seg(p, lo, hi, lane);  // built by the whole warp (shuffles)
+    if (lane == 0) {
+      uint32_t n_blk = 0, n_q = 0, n_seg = 0;
+      bool ok = true;
+      auto tS = [&](uint32_t gb) { return tmem + ((gb & 1) ? kTmS1 : kTmS0); };
+      // S = Q K^T for block gb (nv pages): both operands K-major; k-step kk
+      // starts 32 bytes further into the 128-byte rows, the second 64
+      // features one half further on.
+      auto issue_s = [&](uint32_t gb, uint32_t q_addr, int nv) {
+        const uint32_t stage = s_ring + (gb % kStages) * kStageBytes;
+        const uint64_t a0 = sw128_desc(q_addr, 16, 1024);
+        const uint64_t b0 = sw128_desc(stage, 16, 1024);
+        const uint32_t idesc = make_idesc(1u, 128, nv * kPage, false);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t bk = kk * 32;
+          const uint32_t offa = ((bk / 128) * p.q_half + (bk % 128)) >> 4;
+          const uint32_t offb = ((bk / 128) * kHalf + (bk % 128)) >> 4;
+          mma_f16_ss(tS(gb), a0 + offa, b0 + offb, idesc, kk > 0);
+        }
+      };
+      // O (+)= P V: P from TMEM over S (16 tokens = 8 columns per k-step), V
+      // MN-major with its two 64-feature halves kHalf apart.
+      auto issue_pv = [&](uint32_t gb, int nv, bool acc) {
+        const uint32_t stage = s_ring + (gb % kStages) * kStageBytes;
+        const uint64_t b0 = sw128_desc(stage + 2 * kHalf, kHalf, 1024);
+        for (int kk = 0; kk < nv; ++kk)
+          mma_f16_ts(tmem + kTmO, tS(gb) + kk * 8, b0 + ((kk * kPageHalf) >> 4), kIdescPV,
+                     (acc || kk > 0) ? 1u : 0u);
+      };
+      while (seg.more() && ok) {
+        int b, kvh, pg_lo, pg_hi, P;
+        long long pre;
+        seg.take(b, kvh, pg_lo, pg_hi, pre, P);
+        const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
+        const uint32_t qs = n_q & 1;
+        ok = mbar_wait(&sm.q_full[qs], (n_q >> 1) & 1, g);
+        if (!ok) break;
+        ++n_q;
+        const uint32_t q_addr = s_q + qs * q_slot;
+        for (int j = 0; j < nb && ok; ++j) {
+          const uint32_t gb = n_blk + j;
+          if (j == 0) {
+            ok = mbar_wait(&sm.kv_full[gb % kStages], (gb / kStages) & 1, g);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(gb, q_addr, min(kBlkPages, pg_hi - pg_lo));
+            tc_commit(&sm.s_full[gb & 1]);
+          }
+          if (j + 1 < nb) {  // next block's scores while this block's softmax runs
+            const uint32_t gn = gb + 1;
+            ok = mbar_wait(&sm.kv_full[gn % kStages], (gn / kStages) & 1, g);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(gn, q_addr, min(kBlkPages, pg_hi - (pg_lo + (j + 1) * kBlkPages)));
+            tc_commit(&sm.s_full[gn & 1]);
+          }
+          ok = mbar_wait(&sm.p_full[gb & 1], (gb >> 1) & 1, g);
+          if (!ok) break;
+          if (j == 0 && n_seg > 0) {
+            ok = mbar_wait(&sm.o_empty, (n_seg - 1) & 1, g);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0);
+          tc_commit(&sm.kv_empty[gb % kStages]);
+          tc_commit(&sm.pv_done);
+        }
+        if (!ok) break;
+        tc_commit(&sm.o_full);
+        tc_commit(&sm.q_empty[qs]);
+        n_blk += nb;
+        ++n_seg;
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      tc_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, g_drain);
+    }
+    __syncwarp();
+    finish();
+  } else if (warp < p.sm_warps) {
+    // ------------------------------------------------------------ softmax
+    const int r = warp * 32 + lane;  // query head within the K/V group = TMEM lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t n_blk = 0, n_seg = 0;
+    bool ok = true;
+    Segments seg(p, lo, hi, lane);
+    while (seg.more() && ok) {
+      int b, kvh, pg_lo, pg_hi, P;
+      long long pre;
+      seg.take(b, kvh, pg_lo, pg_hi, pre, P);
+      const int len = len_of(p.seq_lens, p.max_pages, b);
+      const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
+      // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
+      // the MMA multiplies (normalises o so its weights sum to one).
+      float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
+      for (int j = 0; j < nb; ++j) {
+        const uint32_t gb = n_blk + j;
+        const uint32_t tS = tmem + ((gb & 1) ? kTmS1 : kTmS0) + lane_off;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[gb & 1], (gb >> 1) & 1, g));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[kBlkTok];
+        tmem_ld64(tS, sr);
+        const int pg0 = pg_lo + j * kBlkPages;
+        const int nv = pg_hi - pg0 < kBlkPages ? pg_hi - pg0 : kBlkPages;
+        const int tok0 = pg0 * kPage;
+        const int valid = min(nv * kPage, len - tok0);  // tokens of this block that exist
+        if (valid < kBlkTok) {
+#pragma unroll
+          for (int i = 0; i < kBlkTok; ++i)
+            if (i >= valid) sr[i] = 0xFF800000u;  // -inf
+        }
+        float pm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pm[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
+#pragma unroll
+        for (int i0 = 16; i0 < kBlkTok; i0 += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pm[i] = max3(pm[i], __uint_as_float(sr[i0 + i]), __uint_as_float(sr[i0 + 8 + i]));
+        const float mx = fmaxf(max3(pm[0], pm[1], pm[2]), max3(max3(pm[3], pm[4], pm[5]), pm[6], pm[7]));
+        const float m_blk = mx * sl2;
+        float alpha = 1.f;
+        if (m_blk > m_run + kRescaleThreshold) {
+          alpha = ex2_approx(m_run - m_blk);  // m_run = -inf -> 0
+          m_run = m_blk;
+        }
+        l_run *= alpha;
+        l_rnd *= alpha;
+        // Rescale o when the running max moved; the previous block's P V must
+        // have completed first.
+        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (gb - 1) & 1, g));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c4 = 0; c4 < kD / 32; ++c4) {
+            uint32_t raw[32];
+            tmem_ld32(tmem + kTmO + lane_off + c4 * 32, raw);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+            tmem_st32(tmem + kTmO + lane_off + c4 * 32, raw);
+          }
+        }
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
+        uint64_t rs2[4] = {0, 0, 0, 0}, rr2[4] = {0, 0, 0, 0};
+        uint32_t pk[kBlkTok / 2];
+#pragma unroll
+        for (int q2 = 0; q2 < kBlkTok / 2; ++q2) {
+          const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
+          float p0, p1;
+          if ((q2 & 7) >= 6) {  // 2 of every 8 pairs on the FMA pipe
+            f2_split(exp2_poly2(x2), p0, p1);
+          } else {
+            float x0, x1;
+            f2_split(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          rs2[q2 & 3] = add2(rs2[q2 & 3], f2(p0, p1));
+          const uint32_t bb = pack_bf16x2(p0, p1);
+          pk[q2] = bb;
+          rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(bb << 16), __uint_as_float(bb & 0xFFFF0000u)));
+        }
+        {
+          const uint64_t a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
+          const uint64_t bq = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
+          float a0, a1, b0, b1;
+          f2_split(a, a0, a1);
+          f2_split(bq, b0, b1);
+          l_run += a0 + a1;
+          l_rnd += b0 + b1;
+        }
+        tmem_st32(tS, pk);
+        if (warp == 0 && valid < nv * kPage) {
+          // Tokens past the end of the sequence inside its last page: P is 0
+          // there, but the cache slots may hold anything (0 * NaN = NaN), so
+          // their V rows are cleared before the MMA reads them.
+          const uint32_t vst = s_ring + (gb % kStages) * kStageBytes + 2 * kHalf;
+          const int nrow = nv * kPage - valid;  // rows valid .. nv*16-1 of the block
+          for (int e = lane; e < nrow * 2 * 8; e += 32) {
+            const int row = valid + e / 16, h = (e / 8) & 1, ch = e & 7;
+            const uint32_t a = vst + h * kHalf + row * 128 + ch * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[gb & 1]);
+      }
+      if (!ok) break;
+      // End of the segment.
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, n_seg & 1, g));
+      if (!ok) break;
+      tc_fence_after();
+      // One partial per query head.
+      const int sidx = c - owner(pre, T, (int)G);
+      const bool in_range = sidx >= 0 && sidx < p.max_segs;  // always, with chunks >= kDecodeMinChunk
+      if (lane == 0 && !in_range) atomicExch(p.status, kErrBounds);
+      const bool write = r < p.group && in_range;
+      const size_t rec = ((size_t)b * p.Hq + kvh * p.group + r) * p.max_segs + sidx;
+      const float inv = l_rnd > 0.f ? 1.f / l_rnd : 0.f;
+#pragma unroll 1
+      for (int c4 = 0; c4 < kD / 32; ++c4) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + kTmO + lane_off + c4 * 32, raw);
+        if (write) {
+          float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * kD + c4 * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(raw[4 * i]) * inv, __uint_as_float(raw[4 * i + 1]) * inv,
+                                 __uint_as_float(raw[4 * i + 2]) * inv, __uint_as_float(raw[4 * i + 3]) * inv);
+        }
+      }
+      if (write) p.ws_lse[rec] = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_empty);
+      n_blk += nb;
+      ++n_seg;
+    }
+    finish();
+  } else {
+    finish();  // softmax warp without rows (group <= 32 * warp)
+  }
+}
+
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -528,13 +685,13 @@ bool encode_pool(CUtensorMap* map, const void* pool, int num_pages, int Hkv) {
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-// q [B * Hq rows, D] bf16, box = 32 rows x 64 features (128-byte swizzle).
-bool encode_q(CUtensorMap* map, const void* q, int rows) {
+// q [B * Hq rows, D] bf16, box = `box_rows` rows x 64 features (128-byte swizzle).
+bool encode_q(CUtensorMap* map, const void* q, int rows, int box_rows) {
   auto enc = encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kQRows};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -546,30 +703,32 @@ bool encode_q(CUtensorMap* map, const void* q, int rows) {
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (a.D != kD || a.page_size != kPage) return -2;
   const int group = a.Hq / a.Hkv;
-  if (group > 32) return -2;
+  if (group > kMaxGroup) return -2;
   const int max_pages = a.max_pages > 0 ? a.max_pages : 1;
   const int max_segs = decode_max_segments(max_pages);
-  static bool attr_set[64] = {false};
+  const int q_half = (group + 7) / 8 * 8 * 128;
+  const int smem = dec_smem_bytes(q_half);
+  static int attr_smem[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
-  if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (dev >= 64 || attr_smem[dev] < smem) {
+    err = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return fail_cuda("decode: cudaFuncSetAttribute", err);
-    attr_set[dev] = true;
+    if (dev < 64) attr_smem[dev] = smem;
   }
   float* ws_o = static_cast<float*>(a.workspace);
   float* ws_lse = ws_o + (size_t)a.B * a.Hq * max_segs * kD;
-  int* ws_nseg = reinterpret_cast<int*>(ws_lse + (size_t)a.B * a.Hq * max_segs);
   int* status = device_status_word();
   if (!status) return fail_cuda("decode: status word", cudaGetLastError());
-  if (a.num_pages > 0 && a.max_pages > 0) {
+  const int split_grid = kCtasPerSm * sm_count();
+  const bool has_pool = a.num_pages > 0 && a.max_pages > 0;
+  if (has_pool) {
     SplitParams sp{};
     sp.block_table = a.block_table;
     sp.seq_lens = a.seq_lens;
     sp.ws_o = ws_o;
     sp.ws_lse = ws_lse;
-    sp.ws_nseg = ws_nseg;
     sp.B = a.B;
     sp.Hq = a.Hq;
     sp.Hkv = a.Hkv;
@@ -577,23 +736,24 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sp.num_pages = a.num_pages;
     sp.max_pages = a.max_pages;
     sp.max_segs = max_segs;
+    sp.q_half = q_half;
+    sp.sm_warps = (group + 31) / 32;
     sp.scale_log2 = a.scale * kLog2e;
     sp.bounds_check = (debug_flags() & 1) ? 1 : 0;
     sp.status = status;
     sp.timeout_ns = wait_timeout_ns();
     sp.stall = (debug_flags() & 2) ? 1 : 0;
     CUtensorMap tq, tk, tv;
-    if (!encode_q(&tq, a.q, a.B * a.Hq) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
+    if (!encode_q(&tq, a.q, a.B * a.Hq, group) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
         !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv))
       return fail_cuda("decode: tensor map", cudaErrorInvalidValue);
-    decode_split_kernel<<<kCtasPerSm * sm_count(), kThreads, kSmemBytes, stream>>>(tq, tk, tv, sp);
+    decode_split_kernel<<<split_grid, kThreads, smem, stream>>>(tq, tk, tv, sp);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail_cuda("decode: split launch", err);
   }
   CombineParams cp{};
   cp.ws_o = ws_o;
   cp.ws_lse = ws_lse;
-  cp.ws_nseg = ws_nseg;
   cp.seq_lens = a.seq_lens;
   cp.o = static_cast<__nv_bfloat16*>(a.o);
   cp.lse = a.lse;
@@ -603,12 +763,23 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cp.group = group;
   cp.max_pages = max_pages;
   cp.max_segs = max_segs;
-  // Without a pool the split kernel did not run and wrote no segment counts:
-  // the combine then treats every sequence as empty (O = 0, LSE = -inf).
-  cp.has_pool = (a.num_pages > 0 && a.max_pages > 0) ? 1 : 0;
+  cp.split_grid = split_grid;
+  // Without a pool the split kernel did not run: the combine then treats
+  // every sequence as empty (O = 0, LSE = -inf).
+  cp.has_pool = has_pool ? 1 : 0;
   const int nw = a.B * a.Hq;
-  decode_combine_kernel<<<(nw + 7) / 8, 256, 0, stream>>>(cp);
-  err = cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((nw + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, decode_combine_kernel, cp);
+  if (err == cudaSuccess) err = cudaGetLastError();
   return err == cudaSuccess ? 0 : fail_cuda("decode: combine launch", err);
 }
 

@@ -61,11 +61,11 @@ constexpr int kDecodeMinChunk = ATTN_DECODE_MIN_CHUNK;  // pages (512 tokens)
 inline int decode_max_segments(int max_pages) {
   return (max_pages + kDecodeMinChunk - 1) / kDecodeMinChunk + 1;
 }
-// Workspace: partial outputs [B*Hq][S][D] f32, their LSE [B*Hq][S] f32 and the
-// segment count of every (sequence, K/V head) [B*Hq] int32, S = segments.
+// Workspace: partial outputs [B*Hq][S][D] f32 and their log2-sum-exp
+// [B*Hq][S] f32, S = segments.
 inline size_t decode_workspace_bytes(int B, int Hq, int max_pages, int D) {
   const size_t rows = (size_t)B * Hq, segs = (size_t)decode_max_segments(max_pages);
-  return rows * segs * (size_t)(D + 1) * 4 + rows * 4;
+  return rows * segs * (size_t)(D + 1) * 4;
 }
 
 }  // namespace attn

@@ -124,8 +124,9 @@ ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
 /*
  * attn_decode_workspace_bytes -- size of the scratch buffer attn_decode_paged
  * needs for these sizes: per query head of every sequence, up to
- * ceil(max_pages_per_seq / 32) + 1 partial results of D + 1 floats, plus one
- * int per (sequence, query head).  Host only; never fails (0 for empty shapes).
+ * S = ceil(max_pages_per_seq / 32) + 1 partial results of D + 1 floats
+ * (B * Hq * S * (D + 1) * 4 bytes).  Host only; never fails (0 for empty
+ * shapes).
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D);
 
@@ -145,14 +146,20 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq
  *   lse         [B, Hq] fp32 (written; may be NULL)
  *   workspace   caller-owned device scratch of at least
  *               attn_decode_workspace_bytes(B, Hq, max_pages_per_seq, D) bytes;
- *               its contents on entry do not matter.
+ *               its contents on entry do not matter, but two calls that may
+ *               run at the same time must not share one.
  *
  * The single query sees every cached key (causal alignment at the
- * bottom-right corner).  seq_lens[b] == 0 gives O = 0 and LSE = -inf.
- * Supported: page_size == 16, D == 128, Hq % Hkv == 0 and Hq / Hkv <= 32.
+ * bottom-right corner); cache slots past seq_lens[b] in a sequence's last
+ * page are never used, whatever they hold.  seq_lens[b] == 0 gives O = 0 and
+ * LSE = -inf.
+ * Supported: page_size == 16, D == 128, Hq % Hkv == 0 and Hq / Hkv <= 128
+ * (otherwise ATTN_ERR_UNSUPPORTED).
  * Page ids are trusted unless bounds-check mode is on (attn_set_debug), in
- * which case an id outside [0, num_pages) is skipped and reported as
- * ATTN_ERR_BOUNDS by attn_last_device_error().
+ * which case an id outside [0, num_pages) reads as a page of zeros and is
+ * reported as ATTN_ERR_BOUNDS by attn_last_device_error().  Pages are copied
+ * by the tensor-memory-access unit against the pool's bounds, so an untrusted
+ * id cannot make the kernel read outside the pool either way.
  */
 ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                                const int* block_table, const int* seq_lens, void* o, float* lse,

@@ -61,8 +61,9 @@ def test_workspace_size_formula(cdll):
     import attention_flash_attn_02_b200 as attn
     # a sequence of P pages is cut into at most ceil(P / 32) + 1 segments; each
     # leaves D + 1 floats per query head; plus one int per (sequence, head)
-    assert attn.attn_decode_workspace_bytes(64, 32, 512, 128) == 64 * 32 * 17 * 129 * 4 + 64 * 32 * 4
-    assert attn.attn_decode_workspace_bytes(2, 4, 33, 128) == 2 * 4 * 3 * 129 * 4 + 2 * 4 * 4
+    # rows x segments x (D + 1) floats: each partial and its log-sum-exp
+    assert attn.attn_decode_workspace_bytes(64, 32, 512, 128) == 64 * 32 * 17 * 129 * 4
+    assert attn.attn_decode_workspace_bytes(2, 4, 33, 128) == 2 * 4 * 3 * 129 * 4
     assert attn.attn_decode_workspace_bytes(0, 4, 33, 128) == 0
 
 
@@ -124,7 +125,7 @@ def _dec(cdll, **kw):
     (dict(bt=_P(0x10002)), -1),         # misaligned int32 table
     (dict(page=32), -2),                # only 16-token pages are built
     (dict(D=64), -2),
-    (dict(Hq=64, Hkv=1), -2),           # group > 32
+    (dict(Hq=256, Hkv=1), -2),          # group > 128
     (dict(B=0), 0),
 ])
 def test_decode_host_validation(cdll, kw, code):

@@ -177,6 +177,9 @@ def test_decode_full_workload(lib):
     ([700, 1, 64], 16, 2),
     ([5000, 31], 8, 8),
     ([0, 0], 32, 1),
+    ([300, 77, 1], 64, 1),       # two softmax warps per K/V group
+    ([129, 4000], 128, 1),       # four
+    ([50, 33, 16], 12, 4),       # group of 3 (query rows padded to 8)
 ])
 def test_decode_edge_lengths(lib, lens, Hq, Hkv):
     shape = DecodeShape("edge", B=len(lens), Hq=Hq, Hkv=Hkv, D=128, len_lo=1, len_hi=1)
@@ -184,6 +187,28 @@ def test_decode_edge_lengths(lib, lens, Hq, Hkv):
     o, lse = _run_decode(lib, kv, shape.scale)
     o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
     _check(o, o_ref, lse, l_ref, what=str(lens))
+
+
+def test_decode_ignores_cache_slots_past_the_end(lib):
+    # Slots of the last page beyond a sequence's length (and pages no table
+    # entry reaches) hold NaN: attention over the first `len` tokens must not
+    # see them.
+    shape = DecodeShape("nan-tail", B=4, Hq=32, Hkv=2, D=128, len_lo=1, len_hi=1)
+    lens = [17, 100, 1, 250]
+    kv = decode_inputs(shape, 11, seq_lens=lens, extra_pages=3)
+    used = torch.zeros(kv.num_pages, dtype=torch.bool)
+    for b, n in enumerate(lens):
+        npg = (n + 15) // 16
+        used[kv.block_table[b, :npg].long()] = True
+        last = int(kv.block_table[b, npg - 1])
+        kv.k_pages[last, n - (npg - 1) * 16:] = float("nan")
+        kv.v_pages[last, n - (npg - 1) * 16:] = float("nan")
+    kv.k_pages[~used] = float("nan")
+    kv.v_pages[~used] = float("nan")
+    o, lse = _run_decode(lib, kv, shape.scale)
+    o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    _check(o, o_ref, lse, l_ref, what="nan-tail")
 
 
 def test_decode_invariant_to_page_permutation(lib):
