@@ -200,6 +200,7 @@ struct Smem {
   uint64_t drain;
   uint64_t kv_full[12], kv_empty[12];
   uint64_t st_full[2];        // row statistics of a unit written (128 arrivals)
+  uint64_t st_empty[2];       // ... and read by the epilogue (128 arrivals)
   uint32_t tmem_base;
   int abort_flag;
   float st_m[2][kBM];         // [tile][row] running max (log2 units) at unit end
@@ -234,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.o_full[t], 1);
       mbar_init(&sm.o_empty[t], 128);
       mbar_init(&sm.st_full[t], 128);
+      mbar_init(&sm.st_empty[t], 128);
     }
     mbar_init(&sm.drain, 1);
     for (int s = 0; s < C::NS; ++s) {
@@ -299,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = sm.st_m[t][r];
           l = sm.st_l[t][r];
           lr = sm.st_r[t][r];
+          mbar_arrive(&sm.st_empty[t]);  // the softmax may write the next unit's
         }
         const float inv = (lr > 0.f) ? p.out_scale / lr : 0.f;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)w.bh_of(t) * p.Lq + row) * D;
@@ -601,7 +604,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&sm.p_full[t]);
         }
         if (!ok) break;
-        // hand the row statistics of this unit to the epilogue warpgroup
+        // Hand the row statistics of this unit to the epilogue warpgroup, once
+        // it has taken the previous unit's: a unit of one K/V block can finish
+        // while the epilogue is still on the other tile of the unit before.
+        if (nunit > 0) {
+          ok = mbar_wait(&sm.st_empty[t], (nunit - 1) & 1, g);
+          if (!ok) break;
+        }
         sm.st_m[t][r] = m_run;
         sm.st_l[t][r] = l_run;
         sm.st_r[t][r] = l_rnd;
