@@ -43,10 +43,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sources they were taken on (sha256 prefix of the files); a changed kernel
 # reports null until it is captured again.
 PROFILED_TRAFFIC = {
-    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "87167add744fa66f",
-                "bytes": 313_984_000 + 100_759_552, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
-    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "f4e47003e5793c86",
-               "bytes": 147_888_384 + 4_291_328, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
+    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "cf6866cd14575b31",
+                "bytes": 307_631_360 + 97_784_576, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
+    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "498976c04c88a208",
+               "bytes": 147_962_112 + 4_209_664, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
 }
 
 
