@@ -283,36 +283,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  {
-    // Pull this CTA's slice of the block table toward L2 now; the page ids it
-    // will read are only known once the page counts below are summed.
-    const size_t tbytes = (size_t)p.B * p.max_pages * 4;
-    const size_t per = ((tbytes + gridDim.x - 1) / gridDim.x + 127) / 128 * 128;
-    const size_t off = (size_t)blockIdx.x * per + (size_t)tid * 128;
-    if (tid * 128 < per && off < tbytes)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(p.block_table) + off));
-  }
-  // Total pages T of the batch and this CTA's share.  Every warp sums the
-  // page counts itself, lane l taking sequences l, l + 32, ... (independent
-  // loads, then a shuffle reduction), so no warp waits for another.
-  long long T = 0;
-  for (int b = lane; b < p.B; b += 32) T += pages_of(p.seq_lens, p.max_pages, b);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
-  T *= p.Hkv;
-  const long long G = split_ctas(T, gridDim.x);
-  const int c = blockIdx.x;
-  // The combine launch may start now: it waits for this grid's completion
-  // (griddepcontrol.wait) before it reads any partial.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (T == 0 || c >= G) return;
-  const long long lo = c * T / G, hi = (c + 1) * T / G;
-
   const uint32_t base = smem_u32(smem_raw);
   if (base & 1023u) {  // the layout below needs a 1024-byte aligned base
     if (tid == 0) atomicExch(p.status, kErrBounds);
     return;
   }
+  // The page counts of the first 64 sequences are requested before anything
+  // else; barrier set-up and the TMEM allocation run while they are in flight.
+  const int sl0 = lane < p.B ? p.seq_lens[lane] : 0;
+  const int sl1 = lane + 32 < p.B ? p.seq_lens[lane + 32] : 0;
   const uint32_t q_slot = 2u * p.q_half;
   const uint32_t s_q = base;                       // two query slots
   const uint32_t s_ring = base + 2u * q_slot;      // kStages x 32 KB
@@ -339,9 +318,41 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // Total pages T of the batch and this CTA's share.  Every warp sums the
+  // page counts itself, lane l taking sequences l, l + 32, ... (independent
+  // loads, then a shuffle reduction), so no warp waits for another.
+  auto pages_from_len = [&](int n) {
+    const int cap = p.max_pages * kPage;
+    n = n < 0 ? 0 : (n > cap ? cap : n);
+    return (n + kPage - 1) / kPage;
+  };
+  long long T = (long long)pages_from_len(sl0) + pages_from_len(sl1);
+  for (int b = lane + 64; b < p.B; b += 32) T += pages_of(p.seq_lens, p.max_pages, b);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
+  T *= p.Hkv;
+  const long long G = split_ctas(T, gridDim.x);
+  const int c = blockIdx.x;
+  // The combine launch may start now: it waits for this grid's completion
+  // (griddepcontrol.wait) before it reads any partial.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const bool idle = T == 0 || c >= G;
+  const long long lo = idle ? 0 : c * T / G, hi = idle ? 0 : (c + 1) * T / G;
+  if (warp == 4 && !idle) {
+    // Request the first page ids of this CTA's share now, into L1 (the
+    // producer reads them after the barrier below).
+    const Segments s0(p, lo, hi, lane);
+    const int pg = (int)(lo - s0.pre) + lane;
+    if (pg < s0.P)
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(p.block_table + (size_t)s0.b * p.max_pages + pg));
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (idle) {  // no pages for this CTA
+    if (warp == 5) tmem_dealloc(sm.tmem_base, kTmemCols);
+    return;
+  }
   const uint32_t tmem = sm.tmem_base;
   const WaitGuard g{&sm.abort_flag, p.status, p.timeout_ns, true};
   const WaitGuard g_drain{&sm.abort_flag, p.status, p.timeout_ns, false};
