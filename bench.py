@@ -394,6 +394,36 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def fp8_gemm_peak(dev):
+    """Dense e4m3 tensor throughput on this GPU: a cuBLASLt 8192^3 GEMM with
+    fp32 accumulation (torch._scaled_mm, unit scales, bf16 out), best of 10
+    after 3 warm-ups, 2*N^3 FLOP each.  The denominator for the FP8 workload,
+    in the style of the measured bf16 peak; None if the call is unavailable."""
+    import torch
+    n = 8192
+    try:
+        g = torch.Generator(device="cpu").manual_seed(7)
+        a = torch.randn(n, n, generator=g).to(dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, generator=g).to(dev).to(torch.float8_e4m3fn).t()  # column-major operand
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        torch.cuda.empty_cache()
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
+
+
 def side_workloads(attn, dev, peaks, world):
     """Per-launch TFLOP/s of the sliding-window and FP8 workloads (median of
     5 launches after 2 warm-ups; inputs larger than L2)."""
@@ -423,7 +453,13 @@ def side_workloads(attn, dev, peaks, world):
         entry = {"TFLOP/s": round(tf, 1), "ms": round(ms, 3), "bytes_MB": round(prefill_bytes(shape) / 1e6, 1)}
         if shape.fp8:
             entry["frac_of_bf16_peak"] = round(tf / peaks["bf16_tflops"], 4)
-            entry["note"] = "no measured FP8 peak; nominal dense FP8 is 2x bf16"
+            fp8_peak = fp8_gemm_peak(dev)
+            if fp8_peak:
+                entry["fp8_peak_tflops"] = round(fp8_peak, 1)
+                entry["frac_of_fp8_peak"] = round(tf / fp8_peak, 4)
+                entry["fp8_peak_source"] = "measured here: cuBLASLt e4m3 8192^3 GEMM (torch._scaled_mm), best of 10"
+            else:
+                entry["note"] = "FP8 GEMM probe unavailable; nominal dense FP8 is 2x bf16"
         else:
             entry["frac"] = round(tf / peaks["bf16_tflops"], 4)
         out[shape.name] = entry
