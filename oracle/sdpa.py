@@ -232,20 +232,28 @@ def gather_pages(pages, block_table_row, seq_len: int, page_size: int) -> np.nda
 
 
 def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_size: int = 16):
-    """Single-token decode over a paged KV cache.
+    """Decode over a paged KV cache.
 
-    q [B, Hq, D]; pools [num_pages, page_size, Hkv, D]; block_table
-    [B, max_pages]; seq_lens [B].  Each sequence's cache is gathered into the
-    contiguous ``[B, Hkv, seq_len, D]`` view (KV-cache section of p3) and the
-    plain definition is applied with one query row, which sees every cached
-    key.  Returns (O [B, Hq, Dv], LSE [B, Hq]); an empty cache gives O = 0 and
+    q [B, Hq, D] (one new token per sequence) or [B, Hq, q_len, D] (the last
+    q_len tokens of each sequence, e.g. draft tokens to verify); pools
+    [num_pages, page_size, Hkv, D]; block_table [B, max_pages]; seq_lens [B]
+    (cached tokens, the q_len new ones included).  Each sequence's cache is
+    gathered into the contiguous ``[B, Hkv, seq_len, D]`` view (KV-cache
+    section of p3) and the plain definition is applied: with one query row it
+    sees every cached key; with q_len rows, row i is the token at position
+    seq_len - q_len + i and sees the keys up to it (the causal mask aligned at
+    the bottom-right corner).  Returns O [B, Hq, Dv] and LSE [B, Hq] (or
+    [B, Hq, q_len, Dv] and [B, Hq, q_len]); a row without keys gives O = 0 and
     LSE = -inf."""
     q = _f64(q)
-    B, Hq, D = q.shape
+    multi = q.ndim == 4
+    if not multi:
+        q = q[:, :, None, :]
+    B, Hq, Lq, D = q.shape
     lens = [int(x) for x in np.asarray(_f64(seq_lens))]
     Dv = _f64(v_pages[:1]).shape[-1] if len(v_pages) else D
-    out = np.zeros((B, Hq, Dv))
-    lse = np.full((B, Hq), -np.inf)
+    out = np.zeros((B, Hq, Lq, Dv))
+    lse = np.full((B, Hq, Lq), -np.inf)
     kp, vp = _f64(k_pages), _f64(v_pages)
     table = np.asarray(_f64(block_table), dtype=np.int64)
     for b in range(B):
@@ -253,9 +261,11 @@ def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_
         vb = gather_pages(vp, table[b], lens[b], page_size)
         kb = kb.transpose(1, 0, 2)[None]                          # [1, Hkv, len, D]
         vb = vb.transpose(1, 0, 2)[None]
-        o_b, l_b = attention(q[b][None, :, None, :], kb, vb, scale, causal=False)
-        out[b] = o_b[0, :, 0]
-        lse[b] = l_b[0, :, 0]
+        o_b, l_b = attention(q[b][None], kb, vb, scale, causal=multi)
+        out[b] = o_b[0]
+        lse[b] = l_b[0]
+    if not multi:
+        return out[:, :, 0], lse[:, :, 0]
     return out, lse
 
 

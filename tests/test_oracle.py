@@ -316,6 +316,44 @@ def test_paged_decode_empty_sequence():
     assert np.all(np.isfinite(lse[1]))
 
 
+def test_multi_token_decode_rows_equal_truncated_single_token_decode():
+    """Row i of a q_len-token decode is the single-token decode of that token
+    over the cache truncated just after it (len - q_len + i + 1 tokens): the
+    bottom-right causal alignment checked against an independent route."""
+    shape, kv = _small_decode([20, 33, 5, 16], Hq=4, Hkv=2, D=8, seed=52)
+    q_len = 3
+    g = torch.Generator().manual_seed(9)
+    qm = torch.randn(shape.B, shape.Hq, q_len, shape.D, generator=g).to(torch.bfloat16)
+    o, lse = oracle.paged_decode(qm, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3)
+    assert o.shape == (shape.B, shape.Hq, q_len, shape.D) and lse.shape == (shape.B, shape.Hq, q_len)
+    for i in range(q_len):
+        trunc = (kv.seq_lens - q_len + i + 1).clamp(min=0)
+        o1, l1 = oracle.paged_decode(qm[:, :, i], kv.k_pages, kv.v_pages, kv.block_table, trunc, 0.3)
+        np.testing.assert_allclose(o[:, :, i], o1, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, i], l1, rtol=0, atol=1e-13)
+
+
+def test_multi_token_decode_of_one_token_is_single_token_decode():
+    shape, kv = _small_decode([9, 40, 17], seed=53)
+    o1, l1 = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3)
+    o4, l4 = oracle.paged_decode(kv.q[:, :, None], kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3)
+    np.testing.assert_array_equal(o4[:, :, 0], o1)
+    np.testing.assert_array_equal(l4[:, :, 0], l1)
+
+
+def test_multi_token_decode_rows_without_keys():
+    """A cache shorter than q_len leaves the first rows with no key at all:
+    O = 0, LSE = -inf; the last row still sees the whole cache."""
+    shape, kv = _small_decode([2, 6], seed=54)
+    q_len = 4
+    qm = torch.randn(shape.B, shape.Hq, q_len, shape.D, generator=torch.Generator().manual_seed(4))
+    o, lse = oracle.paged_decode(qm, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3)
+    assert np.all(o[0, :, :2] == 0) and np.all(np.isneginf(lse[0, :, :2]))
+    assert np.all(np.isfinite(lse[0, :, 2:])) and np.all(np.isfinite(lse[1]))
+    o1, l1 = oracle.paged_decode(qm[:, :, -1], kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3)
+    np.testing.assert_allclose(o[:, :, -1], o1, rtol=0, atol=1e-13)
+
+
 def test_merge_partials_equals_unsplit():
     """Split the keys into parts, attend each part, merge by LSE: equals
     attention over all keys (float64, to rounding)."""
