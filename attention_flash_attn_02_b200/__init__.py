@@ -64,6 +64,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_decode_workspace_bytes.restype = c_size_t
     lib.attn_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p, c_size_t, c_void_p]
     lib.attn_decode_paged.restype = c_int
+    lib.attn_decode_paged_multi.argtypes = [c_void_p] * 7 + [c_int] * 8 + [c_float, c_void_p, c_size_t, c_void_p]
+    lib.attn_decode_paged_multi.restype = c_int
     lib.attn_decode_paged_noalloc.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p]
     lib.attn_decode_paged_noalloc.restype = c_int
     lib.attn_last_device_error.argtypes = [c_void_p]
@@ -178,6 +180,36 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: Optiona
                                float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _stream_handle(stream))
     _check(st, "attn_decode_paged")
+    return o, lse
+
+
+def attn_decode_paged_multi(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,
+                            o=None, lse=None, workspace=None, stream=None):
+    """Paged decode of the last q_len cached tokens of each sequence (query
+    token i sees the cache up to its own position).  q [B,Hq,q_len,D] bf16;
+    pools, block_table and seq_lens as attn_decode_paged.  Returns
+    (o bf16 [B,Hq,q_len,D], lse fp32 [B,Hq,q_len])."""
+    import torch
+    lib = load()
+    B, Hq, q_len, D = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Hq, q_len, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, q_len), dtype=torch.float32, device=q.device)
+    need = lib.attn_decode_workspace_bytes(B, Hq * q_len, max(max_pages, 1), D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("attn_decode_paged_multi: block_table and seq_lens must be int32")
+    st = lib.attn_decode_paged_multi(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                                     _ptr(o), _ptr(lse), B, Hq, Hkv, q_len, D, page_size, num_pages, max_pages,
+                                     float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream))
+    _check(st, "attn_decode_paged_multi")
     return o, lse
 
 

@@ -114,11 +114,13 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq
   return decode_workspace_bytes(B, Hq, max_pages_per_seq, D);
 }
 
-ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
-                               const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
-                               int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
-                               size_t workspace_bytes, attn_stream_t stream) {
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages_per_seq < 0)
+namespace {
+int decode_checked(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                   const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int q_len, int D,
+                   int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                   size_t workspace_bytes, attn_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages_per_seq < 0 ||
+      q_len <= 0)
     return ATTN_ERR_INVALID;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
   if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;
@@ -129,13 +131,31 @@ ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v
     return ATTN_ERR_INVALID;
   if (num_pages > 0 && (!k_pages || !v_pages || !aligned16(k_pages) || !aligned16(v_pages)))
     return ATTN_ERR_INVALID;
-  if (D != 128 || page_size != 16 || Hq / Hkv > 128) return ATTN_ERR_UNSUPPORTED;
+  if (D != 128 || page_size != 16 || (Hq / Hkv) * q_len > 128) return ATTN_ERR_UNSUPPORTED;
   const int mp = max_pages_per_seq > 0 ? max_pages_per_seq : 1;
-  const size_t need = attn_decode_workspace_bytes(B, Hq, mp, D);
+  const size_t need = attn_decode_workspace_bytes(B, Hq * q_len, mp, D);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_INVALID;
   DecodeArgs a{q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size, num_pages,
-               max_pages_per_seq, scale, workspace, workspace_bytes};
+               max_pages_per_seq, scale, workspace, workspace_bytes, q_len};
   return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                               const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                               int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                               size_t workspace_bytes, attn_stream_t stream) {
+  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, 1, D, page_size,
+                        num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
+}
+
+ATTN_API int attn_decode_paged_multi(const void* q, const void* k_pages, const void* v_pages,
+                                     const int* block_table, const int* seq_lens, void* o, float* lse, int B,
+                                     int Hq, int Hkv, int q_len, int D, int page_size, int num_pages,
+                                     int max_pages_per_seq, float scale, void* workspace, size_t workspace_bytes,
+                                     attn_stream_t stream) {
+  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D, page_size,
+                        num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
 }
 
 ATTN_API int attn_last_device_error(attn_stream_t stream) {

@@ -55,7 +55,7 @@ constexpr int kStageBytes = 4 * kHalf;          // K half 0, K half 1, V half 0,
 constexpr int kCtasPerSm = 2;
 constexpr int kStages = 3;
 constexpr int kThreads = 192;                   // warps 0-3 softmax, 4 producer, 5 MMA
-constexpr int kMaxGroup = 128;                  // query heads per K/V head
+constexpr int kMaxGroup = 128;                  // query rows per K/V head tile: group * q_len
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmS0 = 0, kTmS1 = kBlkTok, kTmO = 2 * kBlkTok;
 static_assert(kTmO + kD <= kTmemCols, "TMEM budget");
@@ -70,8 +70,10 @@ struct SplitParams {
   float* ws_o;    // [B * Hq][S][kD] normalised partial outputs
   float* ws_lse;  // [B * Hq][S] log2-sum-exp of each partial
   int B, Hq, Hkv, group, num_pages, max_pages, max_segs;
+  int q_len;       // query tokens per sequence: the last q_len cached ones
+  int rows;        // query rows per (sequence, K/V head): group * q_len
   int q_half;      // bytes of one 64-feature half of a query tile
-  int sm_warps;    // softmax warps with rows: ceil(group / 32)
+  int sm_warps;    // softmax warps with rows: ceil(rows / 32)
   float scale_log2;
   int bounds_check;
   int* status;
@@ -180,6 +182,7 @@ struct CombineParams {
   __nv_bfloat16* o;
   float* lse;
   int B, Hq, Hkv, group, max_pages, max_segs;
+  int q_len;       // query tokens per sequence
   int split_grid;  // CTAs launched for the split kernel
   int has_pool;    // 0: no page pool, every output is an empty attention
 };
@@ -190,13 +193,13 @@ struct CombineParams {
 // segment s's log2-sum-exp while every lane reads its 4 features of up to 8
 // partials at once.
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);  // output row: (b, h, token)
   const int lane = threadIdx.x & 31;
-  if (gw >= p.B * p.Hq) {
+  if (gw >= p.B * p.Hq * p.q_len) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
-  const int b = gw / p.Hq, h = gw % p.Hq, kvh = h / p.group;
+  const int b = gw / (p.Hq * p.q_len), h = (gw / p.q_len) % p.Hq, kvh = h / p.group;
   int nseg = 0;
   if (p.has_pool) {
     // pages of sequences before b, and in all (seq_lens is an input of the
@@ -385,10 +388,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const uint32_t qs = n_q & 1;
         if (n_q >= 2) ok = mbar_wait(&sm.q_empty[qs], ((n_q >> 1) - 1) & 1, g);
         if (ok) {
-          mbar_arrive_expect_tx(&sm.q_full[qs], 2u * p.group * 128u);
+          mbar_arrive_expect_tx(&sm.q_full[qs], 2u * p.rows * 128u);
           for (int h = 0; h < 2; ++h)
             tma_load_2d(s_q + qs * q_slot + h * p.q_half, &tm_q, &sm.q_full[qs], h * 64,
-                        b * p.Hq + kvh * p.group);
+                        (b * p.Hq + kvh * p.group) * p.q_len);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -521,7 +524,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     finish();
   } else if (warp < p.sm_warps) {
     // ------------------------------------------------------------ softmax
-    const int r = warp * 32 + lane;  // query head within the K/V group = TMEM lane
+    // Row of the group's query tile = TMEM lane: query head r / q_len of the
+    // K/V group, new token r % q_len, which sees the cached tokens up to and
+    // including its own position len - q_len + r % q_len.
+    const int r = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float sl2 = p.scale_log2;
     uint32_t n_blk = 0, n_seg = 0;
@@ -548,10 +554,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int nv = pg_hi - pg0 < kBlkPages ? pg_hi - pg0 : kBlkPages;
         const int tok0 = pg0 * kPage;
         const int valid = min(nv * kPage, len - tok0);  // tokens of this block that exist
-        if (valid < kBlkTok) {
+        const int seen = min(valid, len - p.q_len + r % p.q_len + 1 - tok0);  // ... and this row sees
+        if (seen < kBlkTok) {
 #pragma unroll
           for (int i = 0; i < kBlkTok; ++i)
-            if (i >= valid) sr[i] = 0xFF800000u;  // -inf
+            if (i >= seen) sr[i] = 0xFF800000u;  // -inf
         }
         float pm[8];
 #pragma unroll
@@ -642,8 +649,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const int sidx = c - owner(pre, T, (int)G);
       const bool in_range = sidx >= 0 && sidx < p.max_segs;  // always, with chunks >= kDecodeMinChunk
       if (lane == 0 && !in_range) atomicExch(p.status, kErrBounds);
-      const bool write = r < p.group && in_range;
-      const size_t rec = ((size_t)b * p.Hq + kvh * p.group + r) * p.max_segs + sidx;
+      const bool write = r < p.rows && in_range;
+      const size_t rec = (((size_t)b * p.Hq + kvh * p.group) * p.q_len + r) * p.max_segs + sidx;
       const float inv = l_rnd > 0.f ? 1.f / l_rnd : 0.f;
 #pragma unroll 1
       for (int c4 = 0; c4 < kD / 32; ++c4) {
@@ -714,10 +721,12 @@ bool encode_q(CUtensorMap* map, const void* q, int rows, int box_rows) {
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (a.D != kD || a.page_size != kPage) return -2;
   const int group = a.Hq / a.Hkv;
-  if (group > kMaxGroup) return -2;
+  const int q_len = a.q_len > 0 ? a.q_len : 1;
+  const int rows = group * q_len;  // query rows per (sequence, K/V head) tile
+  if (rows > kMaxGroup) return -2;
   const int max_pages = a.max_pages > 0 ? a.max_pages : 1;
   const int max_segs = decode_max_segments(max_pages);
-  const int q_half = (group + 7) / 8 * 8 * 128;
+  const int q_half = (rows + 7) / 8 * 8 * 128;
   const int smem = dec_smem_bytes(q_half);
   static int attr_smem[64] = {0};
   int dev = 0;
@@ -729,7 +738,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (dev < 64) attr_smem[dev] = smem;
   }
   float* ws_o = static_cast<float*>(a.workspace);
-  float* ws_lse = ws_o + (size_t)a.B * a.Hq * max_segs * kD;
+  float* ws_lse = ws_o + (size_t)a.B * a.Hq * q_len * max_segs * kD;
   int* status = device_status_word();
   if (!status) return fail_cuda("decode: status word", cudaGetLastError());
   const int split_grid = kCtasPerSm * sm_count();
@@ -747,15 +756,17 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sp.num_pages = a.num_pages;
     sp.max_pages = a.max_pages;
     sp.max_segs = max_segs;
+    sp.q_len = q_len;
+    sp.rows = rows;
     sp.q_half = q_half;
-    sp.sm_warps = (group + 31) / 32;
+    sp.sm_warps = (rows + 31) / 32;
     sp.scale_log2 = a.scale * kLog2e;
     sp.bounds_check = (debug_flags() & 1) ? 1 : 0;
     sp.status = status;
     sp.timeout_ns = wait_timeout_ns();
     sp.stall = (debug_flags() & 2) ? 1 : 0;
     CUtensorMap tq, tk, tv;
-    if (!encode_q(&tq, a.q, a.B * a.Hq, group) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
+    if (!encode_q(&tq, a.q, a.B * a.Hq * q_len, rows) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
         !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv))
       return fail_cuda("decode: tensor map", cudaErrorInvalidValue);
     decode_split_kernel<<<split_grid, kThreads, smem, stream>>>(tq, tk, tv, sp);
@@ -774,11 +785,12 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cp.group = group;
   cp.max_pages = max_pages;
   cp.max_segs = max_segs;
+  cp.q_len = q_len;
   cp.split_grid = split_grid;
   // Without a pool the split kernel did not run: the combine then treats
   // every sequence as empty (O = 0, LSE = -inf).
   cp.has_pool = has_pool ? 1 : 0;
-  const int nw = a.B * a.Hq;
+  const int nw = a.B * a.Hq * q_len;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((nw + 7) / 8);
   cfg.blockDim = dim3(256);

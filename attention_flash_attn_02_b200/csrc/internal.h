@@ -33,6 +33,7 @@ struct DecodeArgs {
   float scale;
   void* workspace;
   size_t workspace_bytes;
+  int q_len;  // new tokens per sequence (queries), the last q_len cached ones
 };
 
 // Device status word of the current device (nullptr on failure).

@@ -168,6 +168,33 @@ ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v
                                void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_decode_paged_multi -- attn_decode_paged for q_len new tokens per
+ * sequence (speculative-decoding verification, chunked decode): the last
+ * q_len cached tokens of each sequence are the queries, and query token i
+ * (0-based) sees the cached tokens 0 .. seq_lens[b] - q_len + i (the causal
+ * mask aligned at the bottom-right corner, as in attn_fwd).  Their K/V must
+ * already be in the cache.  (Not a call the pages define: the same
+ * PagedAttention decode with a causal block of queries.)
+ *
+ *   q      [B, Hq, q_len, D] bf16
+ *   o      [B, Hq, q_len, D] bf16 (written)
+ *   lse    [B, Hq, q_len] fp32 (written; may be NULL)
+ *   workspace  at least attn_decode_workspace_bytes(B, Hq * q_len,
+ *              max_pages_per_seq, D) bytes
+ *   everything else as attn_decode_paged.
+ *
+ * A query token with no cached token at or before its position (seq_lens[b]
+ * < q_len) gets O = 0 and LSE = -inf.
+ * Supported: as attn_decode_paged, with (Hq / Hkv) * q_len <= 128 (otherwise
+ * ATTN_ERR_UNSUPPORTED); q_len >= 1 (q_len = 1 is attn_decode_paged).
+ */
+ATTN_API int attn_decode_paged_multi(const void* q, const void* k_pages, const void* v_pages,
+                                     const int* block_table, const int* seq_lens, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int q_len, int D, int page_size, int num_pages,
+                                     int max_pages_per_seq, float scale,
+                                     void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot
  * allocate device memory at the call site (no counterpart in the pages this
  * library follows).

@@ -29,7 +29,7 @@ def _declared_symbols():
 
 def test_header_declares_the_entry_points():
     names = _declared_symbols()
-    for n in ("attn_fwd", "attn_fwd_fp8", "attn_decode_paged", "attn_decode_workspace_bytes",
+    for n in ("attn_fwd", "attn_fwd_fp8", "attn_decode_paged", "attn_decode_paged_multi", "attn_decode_workspace_bytes",
               "attn_last_device_error", "attn_status_str", "attn_set_debug", "attn_version"):
         assert n in names
 
@@ -130,6 +130,26 @@ def _dec(cdll, **kw):
 ])
 def test_decode_host_validation(cdll, kw, code):
     assert _dec(cdll, **kw) == code
+
+
+def _decm(cdll, **kw):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=FAKE, B=2, Hq=32, Hkv=1, q_len=4, D=128,
+             page=16, num_pages=10, max_pages=5, scale=0.1, ws=FAKE, ws_bytes=1 << 22)
+    a.update(kw)
+    return cdll.attn_decode_paged_multi(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["o"], a["lse"], a["B"],
+                                        a["Hq"], a["Hkv"], a["q_len"], a["D"], a["page"], a["num_pages"],
+                                        a["max_pages"], a["scale"], a["ws"], a["ws_bytes"], _P(0))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q_len=0), -1),
+    (dict(q_len=5), -2),                # 32 heads x 5 tokens > 128 rows of one tile
+    (dict(Hq=64, Hkv=2, q_len=4, ws_bytes=16), -1),  # supported (32 x 4 rows): only the workspace stops it
+    (dict(ws_bytes=2 * 32 * 1 * 129 * 4 * 3), -1),  # room for one token per head only
+    (dict(B=0), 0),
+])
+def test_decode_multi_host_validation(cdll, kw, code):
+    assert _decm(cdll, **kw) == code
 
 
 def test_set_debug_returns_previous_flags(cdll):

@@ -15,7 +15,8 @@ import torch
 
 import oracle
 from workloads import (FP8_CAUSAL, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, TINY_MHA, DecodeShape,
-                       PrefillShape, decode_inputs, prefill_inputs, prefill_inputs_fp8, seed_of)
+                       PrefillShape, decode_inputs, decode_queries, prefill_inputs, prefill_inputs_fp8,
+                       seed_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -209,6 +210,51 @@ def test_decode_ignores_cache_slots_past_the_end(lib):
     o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
     _check(o, o_ref, lse, l_ref, what="nan-tail")
+
+
+# ------------------------------------------------------- multi-token decode
+def _run_decode_multi(lib, kv, qm, scale):
+    d = {n: getattr(kv, n).cuda() for n in ("k_pages", "v_pages", "block_table", "seq_lens")}
+    o, lse = lib.attn_decode_paged_multi(qm.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                         scale)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,q_len", [
+    ([100, 17, 1, 2000], 32, 1, 4),      # 128 rows per tile (MQA)
+    ([50, 3, 700, 4096], 32, 8, 8),      # group 4 x 8 tokens
+    ([33, 5000], 8, 2, 2),
+    ([2, 40, 0], 16, 4, 4),              # a cache shorter than q_len: rows without keys
+    ([513, 64], 12, 4, 7),               # group 3 x 7 = 21 rows
+])
+def test_decode_multi_token(lib, lens, Hq, Hkv, q_len):
+    shape = DecodeShape("multi", B=len(lens), Hq=Hq, Hkv=Hkv, D=128, len_lo=1, len_hi=1)
+    kv = decode_inputs(shape, 77 + sum(lens), seq_lens=lens, extra_pages=2)
+    qm = decode_queries(shape, q_len, 78 + q_len)
+    o, lse = _run_decode_multi(lib, kv, qm, shape.scale)
+    o_ref, l_ref = oracle.paged_decode(qm, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, o_ref, lse, l_ref, what=f"{lens} q_len={q_len}")
+
+
+def test_decode_multi_token_full_workload(lib):
+    """The batch-64 MQA cache with 4 new tokens per sequence (all 128 rows of
+    the tile used)."""
+    shape = MQA_DECODE
+    kv = decode_inputs(shape, seed_of(2))
+    qm = decode_queries(shape, 4, seed_of(2) + 100)
+    o, lse = _run_decode_multi(lib, kv, qm, shape.scale)
+    o_ref, l_ref = oracle.paged_decode(qm, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, o_ref, lse, l_ref, what="mqa q_len=4")
+
+
+def test_decode_multi_of_one_token_is_decode(lib):
+    shape = DecodeShape("one", B=5, Hq=32, Hkv=4, D=128, len_lo=10, len_hi=900)
+    kv = decode_inputs(shape, 79)
+    o1, l1 = _run_decode(lib, kv, shape.scale)
+    o2, l2 = _run_decode_multi(lib, kv, kv.q[:, :, None], shape.scale)
+    assert torch.equal(o1, o2[:, :, 0]) and torch.equal(l1, l2[:, :, 0])
 
 
 def test_decode_invariant_to_page_permutation(lib):

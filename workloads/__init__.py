@@ -172,3 +172,10 @@ def decode_inputs(shape: DecodeShape, seed: int, seq_lens: Optional[list] = None
         cursor += npg
     return PagedKV(q=q, k_pages=k_pages, v_pages=v_pages, block_table=table,
                    seq_lens=lens.to(torch.int32))
+
+
+def decode_queries(shape: DecodeShape, q_len: int, seed: int) -> torch.Tensor:
+    """Queries of a q_len-token decode (the last q_len cached tokens of each
+    sequence), [B, Hq, q_len, D] bf16, N(0,1) from their own seed."""
+    g = _gen(seed)
+    return _normal(g, (shape.B, shape.Hq, q_len, shape.D)).to(torch.bfloat16)
