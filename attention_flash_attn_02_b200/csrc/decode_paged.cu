@@ -53,7 +53,7 @@ constexpr int kHalf = kBlkTok * 128;            // a block's 64-feature half (bf
 constexpr int kPageHalf = kPage * 128;          // one page's 64-feature half: 2 KB
 constexpr int kStageBytes = 4 * kHalf;          // K half 0, K half 1, V half 0, V half 1
 constexpr int kCtasPerSm = 2;
-constexpr int kStages = 3;
+constexpr int kMaxStages = 3;                   // ring stages (fewer when the query tile is large)
 constexpr int kThreads = 192;                   // warps 0-3 softmax, 4 producer, 5 MMA
 constexpr int kMaxGroup = 128;                  // query rows per K/V head tile: group * q_len
 constexpr uint32_t kTmemCols = 256;
@@ -73,6 +73,8 @@ struct SplitParams {
   int q_len;       // query tokens per sequence: the last q_len cached ones
   int rows;        // query rows per (sequence, K/V head): group * q_len
   int q_half;      // bytes of one 64-feature half of a query tile
+  int q_slots;     // query tiles in flight (1 or 2)
+  int stages;      // K/V ring stages (2 or 3)
   int sm_warps;    // softmax warps with rows: ceil(rows / 32)
   float scale_log2;
   int bounds_check;
@@ -82,7 +84,7 @@ struct SplitParams {
 };
 
 struct DecSmem {
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done, o_full, o_empty, drain;
@@ -94,10 +96,18 @@ static_assert(sizeof(DecSmem) <= kBarBytes, "barrier block exceeds its reserve")
 // Shared memory: [query slot 0][query slot 1][ring][barriers], the base
 // 1024-byte aligned.  Two CTAs must fit on an SM (233472 bytes, 1 KB of it
 // reserved per CTA) and a third must not (TMEM holds two CTAs' columns).
-__host__ __device__ constexpr int dec_smem_bytes(int q_half) { return 4 * q_half + kStages * kStageBytes + kBarBytes; }
-static_assert(kCtasPerSm * (dec_smem_bytes(32 * 128) + 1024) <= 233472, "the CTAs of an SM must fit");
-static_assert((kCtasPerSm + 1) * (dec_smem_bytes(8 * 128) + 1024) > 233472, "one CTA more must not fit");
-static_assert(dec_smem_bytes(kMaxGroup * 128) <= 232448, "a CTA may use at most 227 KB");
+// Query slots (one or two, each two 64-feature halves) and ring stages are
+// chosen per call so that two CTAs fit on an SM: the deepest ring first, then
+// the second query slot (it only hides the query load at a segment switch).
+__host__ __device__ constexpr int dec_smem_bytes(int q_half, int q_slots, int stages) {
+  return q_slots * 2 * q_half + stages * kStageBytes + kBarBytes;
+}
+constexpr bool two_fit(int bytes) { return kCtasPerSm * (bytes + 1024) <= 233472; }
+static_assert(two_fit(dec_smem_bytes(32 * 128, 2, kMaxStages)), "the MQA tile keeps the full layout");
+static_assert(two_fit(dec_smem_bytes(kMaxGroup * 128, 1, 2)), "the largest tile still fits twice per SM");
+// TMEM holds two CTAs' columns: a launch never asks for so little shared
+// memory that a third CTA would fit on an SM (its allocation would wait).
+constexpr int kMinSmem = 233472 / (kCtasPerSm + 1) - 1024 + 16;
 
 __device__ __forceinline__ int len_of(const int* seq_lens, int max_pages, int b) {
   const int n = seq_lens[b], cap = max_pages * kPage;
@@ -296,11 +306,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int sl0 = lane < p.B ? p.seq_lens[lane] : 0;
   const int sl1 = lane + 32 < p.B ? p.seq_lens[lane + 32] : 0;
   const uint32_t q_slot = 2u * p.q_half;
-  const uint32_t s_q = base;                       // two query slots
-  const uint32_t s_ring = base + 2u * q_slot;      // kStages x 32 KB
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw + 2u * q_slot + kStages * kStageBytes);
+  const uint32_t nqs = (uint32_t)p.q_slots, nst = (uint32_t)p.stages;
+  const uint32_t s_q = base;                       // query slots
+  const uint32_t s_ring = base + nqs * q_slot;     // stages x 32 KB
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw + nqs * q_slot + nst * kStageBytes);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
@@ -385,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       long long pre;
       seg.take(b, kvh, pg_lo, pg_hi, pre, P);
       if (lane == 0) {  // the K/V group's query rows
-        const uint32_t qs = n_q & 1;
-        if (n_q >= 2) ok = mbar_wait(&sm.q_empty[qs], ((n_q >> 1) - 1) & 1, g);
+        const uint32_t qs = n_q % nqs;
+        if (n_q >= nqs) ok = mbar_wait(&sm.q_empty[qs], ((n_q / nqs) - 1) & 1, g);
         if (ok) {
           mbar_arrive_expect_tx(&sm.q_full[qs], 2u * p.rows * 128u);
           for (int h = 0; h < 2; ++h)
@@ -413,8 +424,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
           for (int i = 0; i < kBlkPages; ++i) pid[i] = __shfl_sync(0xffffffffu, id, (kb + i) & 31);
           if (lane == 0) {
-            const uint32_t st = n_blk % kStages;
-            if (n_blk >= (uint32_t)kStages) ok = mbar_wait(&sm.kv_empty[st], ((n_blk / kStages) - 1) & 1, g);
+            const uint32_t st = n_blk % nst;
+            if (n_blk >= nst) ok = mbar_wait(&sm.kv_empty[st], ((n_blk / nst) - 1) & 1, g);
             if (ok) {
               mbar_arrive_expect_tx(&sm.kv_full[st], (uint32_t)nv * 4u * kPageHalf);
               const uint32_t dst = s_ring + st * kStageBytes;
@@ -435,9 +446,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     if (lane == 0) {
       // Drain: the last loads of every slot have landed before the CTA exits.
-      for (uint32_t s = (n_blk > (uint32_t)kStages ? n_blk - kStages : 0); s < n_blk; ++s)
-        mbar_wait(&sm.kv_full[s % kStages], (s / kStages) & 1, g_drain);
-      for (uint32_t s = (n_q > 2u ? n_q - 2 : 0); s < n_q; ++s) mbar_wait(&sm.q_full[s & 1], (s >> 1) & 1, g_drain);
+      for (uint32_t s = (n_blk > nst ? n_blk - nst : 0); s < n_blk; ++s)
+        mbar_wait(&sm.kv_full[s % nst], (s / nst) & 1, g_drain);
+      for (uint32_t s = (n_q > nqs ? n_q - nqs : 0); s < n_q; ++s)
+        mbar_wait(&sm.q_full[s % nqs], (s / nqs) & 1, g_drain);
     }
     finish();
   } else if (warp == 5) {
@@ -451,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       // starts 32 bytes further into the 128-byte rows, the second 64
       // features one half further on.
       auto issue_s = [&](uint32_t gb, uint32_t q_addr, int nv) {
-        const uint32_t stage = s_ring + (gb % kStages) * kStageBytes;
+        const uint32_t stage = s_ring + (gb % nst) * kStageBytes;
         const uint64_t a0 = sw128_desc(q_addr, 16, 1024);
         const uint64_t b0 = sw128_desc(stage, 16, 1024);
         const uint32_t idesc = make_idesc(1u, 128, nv * kPage, false);
@@ -466,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       // O (+)= P V: P from TMEM over S (16 tokens = 8 columns per k-step), V
       // MN-major with its two 64-feature halves kHalf apart.
       auto issue_pv = [&](uint32_t gb, int nv, bool acc) {
-        const uint32_t stage = s_ring + (gb % kStages) * kStageBytes;
+        const uint32_t stage = s_ring + (gb % nst) * kStageBytes;
         const uint64_t b0 = sw128_desc(stage + 2 * kHalf, kHalf, 1024);
         for (int kk = 0; kk < nv; ++kk)
           mma_f16_ts(tmem + kTmO, tS(gb) + kk * 8, b0 + ((kk * kPageHalf) >> 4), kIdescPV,
@@ -477,15 +489,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         long long pre;
         seg.take(b, kvh, pg_lo, pg_hi, pre, P);
         const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
-        const uint32_t qs = n_q & 1;
-        ok = mbar_wait(&sm.q_full[qs], (n_q >> 1) & 1, g);
+        const uint32_t qs = n_q % nqs;
+        ok = mbar_wait(&sm.q_full[qs], (n_q / nqs) & 1, g);
         if (!ok) break;
         ++n_q;
         const uint32_t q_addr = s_q + qs * q_slot;
         for (int j = 0; j < nb && ok; ++j) {
           const uint32_t gb = n_blk + j;
           if (j == 0) {
-            ok = mbar_wait(&sm.kv_full[gb % kStages], (gb / kStages) & 1, g);
+            ok = mbar_wait(&sm.kv_full[gb % nst], (gb / nst) & 1, g);
             if (!ok) break;
             tc_fence_after();
             issue_s(gb, q_addr, min(kBlkPages, pg_hi - pg_lo));
@@ -493,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           }
           if (j + 1 < nb) {  // next block's scores while this block's softmax runs
             const uint32_t gn = gb + 1;
-            ok = mbar_wait(&sm.kv_full[gn % kStages], (gn / kStages) & 1, g);
+            ok = mbar_wait(&sm.kv_full[gn % nst], (gn / nst) & 1, g);
             if (!ok) break;
             tc_fence_after();
             issue_s(gn, q_addr, min(kBlkPages, pg_hi - (pg_lo + (j + 1) * kBlkPages)));
@@ -507,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           }
           tc_fence_after();
           issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0);
-          tc_commit(&sm.kv_empty[gb % kStages]);
+          tc_commit(&sm.kv_empty[gb % nst]);
           tc_commit(&sm.pv_done);
         }
         if (!ok) break;
@@ -626,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           // Tokens past the end of the sequence inside its last page: P is 0
           // there, but the cache slots may hold anything (0 * NaN = NaN), so
           // their V rows are cleared before the MMA reads them.
-          const uint32_t vst = s_ring + (gb % kStages) * kStageBytes + 2 * kHalf;
+          const uint32_t vst = s_ring + (gb % nst) * kStageBytes + 2 * kHalf;
           const int nrow = nv * kPage - valid;  // rows valid .. nv*16-1 of the block
           for (int e = lane; e < nrow * 2 * 8; e += 32) {
             const int row = valid + e / 16, h = (e / 8) & 1, ch = e & 7;
@@ -727,7 +739,17 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int max_pages = a.max_pages > 0 ? a.max_pages : 1;
   const int max_segs = decode_max_segments(max_pages);
   const int q_half = (rows + 7) / 8 * 8 * 128;
-  const int smem = dec_smem_bytes(q_half);
+  int q_slots = 1, stages = 2;  // fits for every tile size (static_assert above)
+  if (two_fit(dec_smem_bytes(q_half, 2, 3))) {
+    q_slots = 2;
+    stages = 3;
+  } else if (two_fit(dec_smem_bytes(q_half, 1, 3))) {
+    stages = 3;
+  } else if (two_fit(dec_smem_bytes(q_half, 2, 2))) {
+    q_slots = 2;
+  }
+  int smem = dec_smem_bytes(q_half, q_slots, stages);
+  if (smem < kMinSmem) smem = kMinSmem;
   static int attr_smem[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -759,6 +781,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sp.q_len = q_len;
     sp.rows = rows;
     sp.q_half = q_half;
+    sp.q_slots = q_slots;
+    sp.stages = stages;
     sp.sm_warps = (rows + 31) / 32;
     sp.scale_log2 = a.scale * kLog2e;
     sp.bounds_check = (debug_flags() & 1) ? 1 : 0;

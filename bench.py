@@ -30,7 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import (FP8_CAUSAL, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, decode_inputs,  # noqa: E402
+from workloads import (FP8_CAUSAL, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, decode_inputs, decode_queries,  # noqa: E402
                        prefill_inputs, prefill_inputs_fp8, seed_of)
 from workloads.accounting import decode_bytes, prefill_bytes, prefill_flops  # noqa: E402
 
@@ -465,7 +465,44 @@ def side_workloads(attn, dev, peaks, world):
         out[shape.name] = entry
         del fn
         torch.cuda.empty_cache()
+    out.update(multi_token_decode(attn, dev, peaks, world))
     return out
+
+
+def multi_token_decode(attn, dev, peaks, world, q_len: int = 4):
+    """GB/s of the batch-64 MQA decode with q_len new tokens per sequence
+    (attn_decode_paged_multi): every page read once for all q_len tokens.
+    L2 flushed (write, then read 256 MB) before each call; median of 10."""
+    import torch
+    kv = decode_inputs(DECODE, seed_of(2))
+    qm = decode_queries(DECODE, q_len, seed_of(2) + 100).to(dev)
+    kp, vp, bt, sl = kv.k_pages.to(dev), kv.v_pages.to(dev), kv.block_table.to(dev), kv.seq_lens.to(dev)
+    o = torch.empty_like(qm)
+    lse = torch.empty(qm.shape[:3], dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.attn_decode_workspace_bytes(DECODE.B, DECODE.Hq * q_len, kv.max_pages, DECODE.D),
+                     dtype=torch.uint8, device=dev)
+    fw = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fr = torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fn = lambda: attn.attn_decode_paged_multi(qm, kp, vp, bt, sl, DECODE.scale, o=o, lse=lse, workspace=ws)  # noqa
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(10):
+        fw.zero_()
+        fr.view(torch.int32).sum(dtype=torch.int32)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = max_over_ranks(statistics.median(ts), world, dev)
+    by = decode_bytes(DECODE, kv.seq_lens.tolist(), q_len)
+    gbs = by / (ms / 1e3) / 1e9
+    return {f"{DECODE.name}_qlen{q_len}": {"GB/s": round(gbs, 1), "us_per_call": round(ms * 1e3, 2),
+                                            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                            "bytes_MB": round(by / 1e6, 1)}}
 
 
 # ------------------------------------------------------------- reference

@@ -39,16 +39,16 @@ def prefill_bytes(shape: PrefillShape) -> float:
     return float(q + kv + o + lse)
 
 
-def decode_bytes(shape: DecodeShape, seq_lens) -> float:
-    """Algorithmic HBM bytes of one paged decode: every cached K and V element
-    of every sequence once, plus q, o, lse, the used block-table entries and
-    seq_lens."""
+def decode_bytes(shape: DecodeShape, seq_lens, q_len: int = 1) -> float:
+    """Algorithmic HBM bytes of one paged decode of q_len tokens per sequence:
+    every cached K and V element of every sequence once, plus q, o, lse, the
+    used block-table entries and seq_lens."""
     ps = shape.page_size
     lens = [int(x) for x in seq_lens]
     kv = sum(lens) * shape.Hkv * shape.D * 2 * 2
-    q = shape.B * shape.Hq * shape.D * 2
-    o = shape.B * shape.Hq * shape.D * 2
-    lse = shape.B * shape.Hq * 4
+    q = shape.B * shape.Hq * q_len * shape.D * 2
+    o = shape.B * shape.Hq * q_len * shape.D * 2
+    lse = shape.B * shape.Hq * q_len * 4
     table = sum((n + ps - 1) // ps for n in lens) * 4 + shape.B * 4
     return float(kv + q + o + lse + table)
 
