@@ -33,6 +33,7 @@ from .sdpa import (  # noqa: F401
     kv_cache_bytes,
     merge_partials,
     online_softmax_attention,
+    kv_append,
     paged_decode,
     repeat_kv,
     visible_key_range,

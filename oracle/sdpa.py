@@ -231,6 +231,32 @@ def gather_pages(pages, block_table_row, seq_len: int, page_size: int) -> np.nda
     return flat[:seq_len]
 
 
+def kv_append(k_pages, v_pages, block_table, seq_lens, k_new, v_new, page_size: int = 16):
+    """Write the K/V of each sequence's newest tokens into its pages.
+
+    k_new, v_new [B, Hkv, L_new, D]; seq_lens [B] counts the cached tokens
+    with the new ones included, so token t of sequence b goes to position
+    ``seq_lens[b] - L_new + t``: page ``block_table[b, pos // page_size]``,
+    slot ``pos % page_size`` (the KV-cache layout of the PagedAttention
+    section of p3).  Positions below 0 are skipped.  Returns new pools
+    (float64); nothing else of the pools changes."""
+    kp = _f64(k_pages).copy()
+    vp = _f64(v_pages).copy()
+    kn, vn = _f64(k_new), _f64(v_new)
+    table = np.asarray(_f64(block_table), dtype=np.int64)
+    B, Hkv, Ln, D = kn.shape
+    for b in range(B):
+        n = int(np.asarray(_f64(seq_lens))[b])
+        for t in range(Ln):
+            pos = n - Ln + t
+            if pos < 0:
+                continue
+            page = table[b, pos // page_size]
+            kp[page, pos % page_size] = kn[b, :, t]
+            vp[page, pos % page_size] = vn[b, :, t]
+    return kp, vp
+
+
 def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_size: int = 16):
     """Decode over a paged KV cache.
 

@@ -354,6 +354,46 @@ def test_multi_token_decode_rows_without_keys():
     np.testing.assert_allclose(o[:, :, -1], o1, rtol=0, atol=1e-13)
 
 
+def test_kv_append_then_decode_equals_contiguous_attention():
+    """Append a chunk of new tokens to paged caches, then attend the chunk's
+    queries over the cache: equals plain causal attention over the
+    contiguous sequence (cached prefix + chunk), bottom-right aligned."""
+    g = torch.Generator().manual_seed(11)
+    B, Hq, Hkv, D, Ln = 3, 4, 2, 8, 5
+    prefix = [7, 16, 0]
+    lens = [n + Ln for n in prefix]
+    shape = DecodeShape("t", B=B, Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=1)
+    kv = decode_inputs(shape, 60, seq_lens=lens, extra_pages=2)
+    k_new = torch.randn(B, Hkv, Ln, D, generator=g)
+    v_new = torch.randn(B, Hkv, Ln, D, generator=g)
+    q = torch.randn(B, Hq, Ln, D, generator=g)
+    kp, vp = oracle.kv_append(kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, k_new, v_new)
+    o, lse = oracle.paged_decode(q, kp, vp, kv.block_table, kv.seq_lens, 0.3)
+    for b in range(B):
+        pre_k = oracle.gather_pages(kv.k_pages, kv.block_table[b], prefix[b], 16).transpose(1, 0, 2)
+        pre_v = oracle.gather_pages(kv.v_pages, kv.block_table[b], prefix[b], 16).transpose(1, 0, 2)
+        kb = np.concatenate([pre_k, k_new[b].double().numpy()], axis=1)[None]
+        vb = np.concatenate([pre_v, v_new[b].double().numpy()], axis=1)[None]
+        ob, lb = _brute(q[b][None].double().numpy(), kb, vb, 0.3, True, 0)
+        np.testing.assert_allclose(o[b], ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=1e-12)
+
+
+def test_kv_append_touches_only_the_new_slots():
+    shape, kv = _small_decode([20, 3], Hq=4, Hkv=2, D=8, seed=61)
+    Ln = 4
+    k_new = torch.randn(2, 2, Ln, 8, generator=torch.Generator().manual_seed(5))
+    kp, vp = oracle.kv_append(kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, k_new, k_new)
+    changed = np.argwhere(np.any(kp != kv.k_pages.double().numpy(), axis=(2, 3)))
+    expect = set()
+    for b, n in enumerate(kv.seq_lens.tolist()):
+        for t in range(Ln):
+            pos = n - Ln + t
+            if pos >= 0:
+                expect.add((int(kv.block_table[b, pos // 16]), pos % 16))
+    assert {tuple(x) for x in changed} <= expect and len(expect) > 0
+
+
 def test_merge_partials_equals_unsplit():
     """Split the keys into parts, attend each part, merge by LSE: equals
     attention over all keys (float64, to rounding)."""
