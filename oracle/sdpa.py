@@ -257,7 +257,7 @@ def kv_append(k_pages, v_pages, block_table, seq_lens, k_new, v_new, page_size: 
     return kp, vp
 
 
-def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_size: int = 16):
+def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_size: int = 16, window: int = 0):
     """Decode over a paged KV cache.
 
     q [B, Hq, D] (one new token per sequence) or [B, Hq, q_len, D] (the last
@@ -268,9 +268,11 @@ def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_
     section of p3) and the plain definition is applied: with one query row it
     sees every cached key; with q_len rows, row i is the token at position
     seq_len - q_len + i and sees the keys up to it (the causal mask aligned at
-    the bottom-right corner).  Returns O [B, Hq, Dv] and LSE [B, Hq] (or
-    [B, Hq, q_len, Dv] and [B, Hq, q_len]); a row without keys gives O = 0 and
-    LSE = -inf."""
+    the bottom-right corner); ``window`` > 0 further limits every row to its
+    last ``window`` keys (sliding window of p3).  Returns O [B, Hq, Dv] and
+    LSE [B, Hq] (or [B, Hq, q_len, Dv] and [B, Hq, q_len]); a row without keys
+    gives O = 0 and LSE = -inf.  The same call defines chunked prefill over
+    a paged cache (q_len in the hundreds or thousands)."""
     q = _f64(q)
     multi = q.ndim == 4
     if not multi:
@@ -287,7 +289,7 @@ def paged_decode(q, k_pages, v_pages, block_table, seq_lens, scale: float, page_
         vb = gather_pages(vp, table[b], lens[b], page_size)
         kb = kb.transpose(1, 0, 2)[None]                          # [1, Hkv, len, D]
         vb = vb.transpose(1, 0, 2)[None]
-        o_b, l_b = attention(q[b][None], kb, vb, scale, causal=multi)
+        o_b, l_b = attention(q[b][None], kb, vb, scale, causal=multi or window > 0, window=window)
         out[b] = o_b[0]
         lse[b] = l_b[0]
     if not multi:

@@ -394,6 +394,20 @@ def test_kv_append_touches_only_the_new_slots():
     assert {tuple(x) for x in changed} <= expect and len(expect) > 0
 
 
+def test_paged_window_equals_contiguous_window():
+    """A sliding window over the paged cache equals the contiguous windowed
+    attention of the gathered sequence (bottom-right aligned)."""
+    shape, kv = _small_decode([30, 47], Hq=4, Hkv=2, D=8, seed=62)
+    q = torch.randn(2, 4, 6, 8, generator=torch.Generator().manual_seed(8))
+    o, lse = oracle.paged_decode(q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3, window=5)
+    for b, n in enumerate(kv.seq_lens.tolist()):
+        kb = oracle.gather_pages(kv.k_pages, kv.block_table[b], n, 16).transpose(1, 0, 2)[None]
+        vb = oracle.gather_pages(kv.v_pages, kv.block_table[b], n, 16).transpose(1, 0, 2)[None]
+        ob, lb = _brute(q[b][None].double().numpy(), kb, vb, 0.3, True, 5)
+        np.testing.assert_allclose(o[b], ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=1e-12)
+
+
 def test_merge_partials_equals_unsplit():
     """Split the keys into parts, attend each part, merge by LSE: equals
     attention over all keys (float64, to rounding)."""
