@@ -66,6 +66,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_decode_paged.restype = c_int
     lib.attn_decode_paged_multi.argtypes = [c_void_p] * 7 + [c_int] * 8 + [c_float, c_void_p, c_size_t, c_void_p]
     lib.attn_decode_paged_multi.restype = c_int
+    lib.attn_prefill_paged.argtypes = [c_void_p] * 7 + [c_int] * 8 + [c_float, c_int, c_void_p]
+    lib.attn_prefill_paged.restype = c_int
+    lib.attn_kv_append.argtypes = [c_void_p] * 6 + [c_int] * 7 + [c_void_p]
+    lib.attn_kv_append.restype = c_int
     lib.attn_decode_paged_noalloc.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p]
     lib.attn_decode_paged_noalloc.restype = c_int
     lib.attn_last_device_error.argtypes = [c_void_p]
@@ -211,6 +215,49 @@ def attn_decode_paged_multi(q, k_pages, v_pages, block_table, seq_lens, scale: O
                                      _stream_handle(stream))
     _check(st, "attn_decode_paged_multi")
     return o, lse
+
+
+def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None, window: int = 0,
+                       o=None, lse=None, stream=None):
+    """Chunked prefill over a paged cache: the last Lq cached tokens of each
+    sequence attend causally to the cache.  q [B,Hq,Lq,D] bf16; pools
+    [P,16,Hkv,D] bf16; block_table [B,max_pages] int32; seq_lens [B] int32.
+    Returns (o bf16 [B,Hq,Lq,D], lse fp32 [B,Hq,Lq])."""
+    import torch
+    lib = load()
+    B, Hq, Lq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Hq, Lq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("attn_prefill_paged: block_table and seq_lens must be int32")
+    st = lib.attn_prefill_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), _ptr(o),
+                                _ptr(lse), B, Hq, Hkv, Lq, D, page_size, num_pages, max_pages, float(scale),
+                                int(window), _stream_handle(stream))
+    _check(st, "attn_prefill_paged")
+    return o, lse
+
+
+def attn_kv_append(k_new, v_new, k_pages, v_pages, block_table, seq_lens, stream=None):
+    """Write k_new/v_new [B,Hkv,L_new,D] bf16 into the pools at positions
+    seq_lens[b] - L_new + t (in place)."""
+    import torch
+    lib = load()
+    B, Hkv, L_new, D = k_new.shape
+    num_pages, page_size, _, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("attn_kv_append: block_table and seq_lens must be int32")
+    st = lib.attn_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                            _ptr(seq_lens), B, Hkv, L_new, D, page_size, num_pages, max_pages,
+                            _stream_handle(stream))
+    _check(st, "attn_kv_append")
+    return k_pages, v_pages
 
 
 def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,

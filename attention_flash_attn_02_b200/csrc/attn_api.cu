@@ -158,6 +158,43 @@ ATTN_API int attn_decode_paged_multi(const void* q, const void* k_pages, const v
                         num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
 }
 
+ATTN_API int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                                const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Lq, int D,
+                                int page_size, int num_pages, int max_pages_per_seq, float scale, int window,
+                                attn_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || D <= 0 || page_size <= 0 || num_pages <= 0 ||
+      max_pages_per_seq <= 0)
+    return ATTN_ERR_INVALID;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
+  if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;
+  if (B == 0) return ATTN_OK;
+  if (!q || !o || !k_pages || !v_pages || !block_table || !seq_lens) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(k_pages) || !aligned16(v_pages)) return ATTN_ERR_INVALID;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID;
+  if ((D != 64 && D != 128) || page_size != 16) return ATTN_ERR_UNSUPPORTED;
+  PrefillArgs a{q, k_pages, v_pages, o, lse, B, Hq, Hkv, Lq, 0, D, scale, 1, window > 0 ? window : 0, false,
+                1.f, 1.f, 1.f, true, block_table, seq_lens, num_pages, max_pages_per_seq};
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+ATTN_API int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                            const int* block_table, const int* seq_lens, int B, int Hkv, int L_new, int D,
+                            int page_size, int num_pages, int max_pages_per_seq, attn_stream_t stream) {
+  if (B < 0 || Hkv <= 0 || L_new < 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages_per_seq < 0)
+    return ATTN_ERR_INVALID;
+  if (B == 0 || L_new == 0) return ATTN_OK;
+  if (num_pages == 0 || max_pages_per_seq == 0) return ATTN_ERR_INVALID;  // nowhere to write
+  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !seq_lens) return ATTN_ERR_INVALID;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pages) || !aligned16(v_pages)) return ATTN_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID;
+  if (D % 8 != 0 || page_size != 16) return ATTN_ERR_UNSUPPORTED;
+  return launch_kv_append(k_new, v_new, k_pages, v_pages, block_table, seq_lens, B, Hkv, L_new, D, num_pages,
+                          max_pages_per_seq, static_cast<cudaStream_t>(stream));
+}
+
 ATTN_API int attn_last_device_error(attn_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
   int* p = device_status_word();

@@ -19,6 +19,12 @@ struct PrefillArgs {
   int causal, window;
   bool fp8;
   float q_descale, k_descale, v_descale;
+  // Paged K/V (chunked prefill over a paged cache): k, v are the page pools
+  // [num_pages, 16, Hkv, D]; Lk is unused (each sequence has seq_lens[b]).
+  bool paged;
+  const int* block_table;
+  const int* seq_lens;
+  int num_pages, max_pages;
 };
 
 struct DecodeArgs {
@@ -49,6 +55,10 @@ int fail_cuda(const char* where, cudaError_t err);
 
 // Launchers: return a status code of include/attn.h.
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+// New tokens' K/V into their slots of the page pools (KV append).
+int launch_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages, const int* block_table,
+                     const int* seq_lens, int B, int Hkv, int L_new, int D, int num_pages, int max_pages,
+                     cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
 // Decode work partition.  Every CTA streams a contiguous share of all cached

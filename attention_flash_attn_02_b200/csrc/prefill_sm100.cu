@@ -109,7 +109,15 @@ struct Params {
   int* status;
   unsigned long long timeout_ns;
   int stall;  // testing hook: the producer issues no loads, every wait runs out
+  // Paged K/V (chunked prefill over a paged cache): sequence b has
+  // seq_lens[b] cached tokens (its Lq queries are the last Lq of them),
+  // stored in 16-token pages of a pool listed by block_table.
+  const int* block_table;
+  const int* seq_lens;
+  int max_pages, num_pages;
 };
+
+constexpr int kPage = 16;  // tokens per page of a paged K/V pool
 
 struct Unit {
   int bh[2];  // b * Hq + head of each tile
@@ -117,6 +125,7 @@ struct Unit {
   int kvbh;   // b * Hkv + kv head
   int kb_lo;  // first K/V block
   int nb;     // number of K/V blocks (0: nothing visible)
+  int lk;     // keys of this unit's sequence (Lk, or its cached length when paged)
   // Per-tile fields by a runtime tile index, as selects (an indexed load
   // would put the struct in local memory).
   __device__ __forceinline__ int bh_of(int t) const { return t ? bh[1] : bh[0]; }
@@ -125,14 +134,14 @@ struct Unit {
 
 // Visible keys [lo, hi) of query row i (bottom-right causal alignment; window
 // of W keys including the query's own position).
-__device__ __forceinline__ void key_range(int i, const Params& p, int& lo, int& hi) {
+__device__ __forceinline__ void key_range(int i, int lk, const Params& p, int& lo, int& hi) {
   if (!p.causal) {
     lo = 0;
-    hi = p.Lk;
+    hi = lk;
     return;
   }
-  int h = i + (p.Lk - p.Lq) + 1;
-  h = h < 0 ? 0 : (h > p.Lk ? p.Lk : h);
+  int h = i + (lk - p.Lq) + 1;
+  h = h < 0 ? 0 : (h > lk ? lk : h);
   hi = h;
   lo = (p.window > 0 && h - p.window > 0) ? h - p.window : 0;
 }
@@ -141,23 +150,32 @@ __device__ __forceinline__ void key_range(int i, const Params& p, int& lo, int& 
 // come first.  CTA c takes one unit per round, in snake order (c in even
 // rounds, grid - 1 - c in odd rounds), which balances the causal work across
 // CTAs to within a fraction of a percent without any global queue.
+template <bool PAGED>
 __device__ __forceinline__ Unit get_unit(int u, const Params& p) {
   Unit w;
+  int b_seq;
   const int mg = p.n_mgroups - 1 - u / p.n_pairs;
   const int pr = u % p.n_pairs;
   if (p.pair_heads) {
     const int hp_per_b = p.Hq >> 1;
     const int b = pr / hp_per_b, hp = pr % hp_per_b;
+    b_seq = b;
     w.bh[0] = b * p.Hq + 2 * hp;
     w.bh[1] = w.bh[0] + 1;
     w.m0[0] = w.m0[1] = mg * kBM;
     w.kvbh = b * p.Hkv + (2 * hp) / p.group;
   } else {
     const int b = pr / p.Hq, h = pr % p.Hq;
+    b_seq = b;
     w.bh[0] = w.bh[1] = b * p.Hq + h;
     w.m0[0] = mg * 2 * kBM;
     w.m0[1] = w.m0[0] + kBM;
     w.kvbh = b * p.Hkv + h / p.group;
+  }
+  w.lk = p.Lk;
+  if (PAGED) {
+    const int n = p.seq_lens[b_seq], cap = p.max_pages * kPage;
+    w.lk = n < 0 ? 0 : (n > cap ? cap : n);
   }
   int lo = INT_MAX, hi = 0;
 #pragma unroll
@@ -165,8 +183,8 @@ __device__ __forceinline__ Unit get_unit(int u, const Params& p) {
     if (w.m0[t] < p.Lq) {
       const int r_last = min(w.m0[t] + kBM - 1, p.Lq - 1);
       int lo0, hi0, lo1, hi1;
-      key_range(w.m0[t], p, lo0, hi0);
-      key_range(r_last, p, lo1, hi1);
+      key_range(w.m0[t], w.lk, p, lo0, hi0);
+      key_range(r_last, w.lk, p, lo1, hi1);
       if (hi1 > lo0) {  // lo and hi are non-decreasing in the row index
         lo = min(lo, lo0);
         hi = max(hi, hi1);
@@ -210,7 +228,7 @@ struct Smem {
 
 static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserve");
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -289,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t nunit = 0;
     bool ok = true;
     for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
-      const Unit w = get_unit(u, p);
+      const Unit w = get_unit<PAGED>(u, p);
       for (int t = 0; t < 2 && ok; ++t) {
         const int row = w.m0_of(t) + r;
         const bool row_valid = row < p.Lq;
@@ -342,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t seq = 0, nunit = 0;
       bool ok = !p.stall;
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
-        const Unit w = get_unit(u, p);
+        const Unit w = get_unit<PAGED>(u, p);
         if (w.nb <= 0) continue;
         for (int t = 0; t < 2 && ok; ++t) {
           if (nunit > 0) ok = mbar_wait(&sm.q_empty[t], (nunit - 1) & 1, g);
@@ -363,9 +381,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = kv_addr0 + s * C::TILE_BYTES;
             mbar_arrive_expect_tx(&sm.kv_full[s], C::TILE_BYTES);
             const CUtensorMap* m = kind == 0 ? &tm_k : &tm_v;
+            if (PAGED) {
+              // The block's 128 keys are 8 pages of this K/V head, gathered
+              // through the block table into the rows of one tile; pages past
+              // the sequence read as zeros (a page id past the pool).
+              const int b = w.kvbh / p.Hkv, kvh = w.kvbh % p.Hkv;
+              const int npg = (w.lk + kPage - 1) / kPage;
+              int ids[kBN / kPage];
 #pragma unroll
-            for (int bx = 0; bx < C::NBOX; ++bx)
-              tma_load_3d(dst + bx * C::BOX_BYTES, m, &sm.kv_full[s], bx * C::BOX_ELEMS, row, w.kvbh);
+              for (int i = 0; i < kBN / kPage; ++i) {
+                const int pg = row / kPage + i;
+                ids[i] = pg < npg ? p.block_table[(size_t)b * p.max_pages + pg] : p.num_pages;
+              }
+#pragma unroll
+              for (int i = 0; i < kBN / kPage; ++i)
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                  tma_load_3d(dst + bx * C::BOX_BYTES + i * (kPage * 128), m, &sm.kv_full[s], bx * C::BOX_ELEMS,
+                              kvh, ids[i] * kPage);
+            } else {
+#pragma unroll
+              for (int bx = 0; bx < C::NBOX; ++bx)
+                tma_load_3d(dst + bx * C::BOX_BYTES, m, &sm.kv_full[s], bx * C::BOX_ELEMS, row, w.kvbh);
+            }
             ++seq;
           }
         }
@@ -421,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
-        const Unit w = get_unit(u, p);
+        const Unit w = get_unit<PAGED>(u, p);
         if (w.nb <= 0) continue;
         ok = mbar_wait(&sm.q_full[0], nunit & 1, g) && mbar_wait(&sm.q_full[1], nunit & 1, g);
         if (!ok) break;
@@ -441,6 +479,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&sm.kv_full[sv], (seq / C::NS) & 1, g);
           if (!ok) break;
           ++seq;
+          if (PAGED) {
+            // Cache slots past the sequence end inside its last page: P is 0
+            // there, but the slots may hold anything (0 * NaN = NaN), so their
+            // V rows are cleared before P V reads them.
+            const int key0 = (w.kb_lo + j) * kBN;
+            const int r_lo = w.lk - key0, r_hi = min((w.lk + kPage - 1) / kPage * kPage - key0, kBN);
+            if (r_lo > 0 && r_lo < r_hi) {
+              for (int rr = r_lo; rr < r_hi; ++rr)
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX; ++bx)
+#pragma unroll
+                  for (int ch = 0; ch < 8; ++ch)
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                     kv_addr0 + sv * C::TILE_BYTES + bx * C::BOX_BYTES + rr * 128 + ch * 16),
+                                 "r"(0u)
+                                 : "memory");
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+          }
           const bool has_next = j + 1 < w.nb;
           const uint32_t skn = seq % C::NS;
           for (int t = 0; t < 2 && ok; ++t) {
@@ -494,14 +551,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t scnt = 0, nunit = 0;
     bool ok = true;
     for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
-      const Unit w = get_unit(u, p);
+      const Unit w = get_unit<PAGED>(u, p);
       const int row = w.m0_of(t) + r;
       // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
       // the MMA multiplies (normalises O so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
       if (w.nb > 0) {
         int lo, hi;
-        key_range(row, p, lo, hi);
+        key_range(row, w.lk, p, lo, hi);
         for (int j = 0; j < w.nb; ++j) {
           ok = mbar_wait(&sm.s_full[t], scnt & 1, g);
           if (!ok) break;
@@ -651,7 +708,22 @@ bool encode_3d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uin
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8>
+// The K/V page pool [num_pages * 16 tokens, Hkv, D] as a 3-D tensor, box =
+// one page of one K/V head, 128 bytes of features (128-byte swizzle).
+bool encode_pool(CUtensorMap* map, const void* pool, bool fp8, int D, int num_pages, int Hkv) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  const uint64_t el = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)num_pages * kPage};
+  cuuint64_t strides[2] = {(cuuint64_t)D * el, (cuuint64_t)Hkv * D * el};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / el), 1, (cuuint32_t)kPage};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool FP8, bool PAGED>
 int run(const PrefillArgs& a, cudaStream_t stream) {
   using C = Cfg<D, FP8>;
   static bool attr_set[64] = {false};
@@ -659,7 +731,8 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
   if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(prefill_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    err = cudaFuncSetAttribute(prefill_kernel<D, FP8, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES);
     if (err != cudaSuccess) return fail_cuda("prefill: cudaFuncSetAttribute", err);
     attr_set[dev] = true;
   }
@@ -690,8 +763,22 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   if (!p.status) return fail_cuda("prefill: status word", cudaGetLastError());
   p.timeout_ns = wait_timeout_ns();
   p.stall = (debug_flags() & 2) ? 1 : 0;
+  p.block_table = a.block_table;
+  p.seq_lens = a.seq_lens;
+  p.max_pages = a.max_pages;
+  p.num_pages = a.num_pages;
 
   CUtensorMap tq, tk, tv;
+  if (PAGED) {
+    if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq))
+      return fail_cuda("prefill: tensor map (q)", cudaErrorInvalidValue);
+    if (!encode_pool(&tk, a.k, FP8, D, a.num_pages, a.Hkv) || !encode_pool(&tv, a.v, FP8, D, a.num_pages, a.Hkv))
+      return fail_cuda("prefill: tensor map (pool)", cudaErrorInvalidValue);
+    const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+    prefill_kernel<D, FP8, PAGED><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    err = cudaGetLastError();
+    return err == cudaSuccess ? 0 : fail_cuda("prefill (paged): launch", err);
+  }
   const bool have_k = a.Lk > 0;
   if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq)) return fail_cuda("prefill: tensor map (q)", cudaErrorInvalidValue);
   // With no keys nothing is loaded from K/V; describe Q instead of an empty tensor.
@@ -700,7 +787,7 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   if (!encode_3d(&tv, have_k ? a.v : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
     return fail_cuda("prefill: tensor map (v)", cudaErrorInvalidValue);
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
-  prefill_kernel<D, FP8><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, FP8, PAGED><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   err = cudaGetLastError();
   return err == cudaSuccess ? 0 : fail_cuda("prefill: launch", err);
 }
@@ -708,12 +795,18 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
 }  // namespace
 
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
-  if (a.fp8) {
-    if (a.D == 128) return run<128, true>(a, stream);
+  if (a.paged) {  // bf16 pools only
+    if (a.fp8) return -2;
+    if (a.D == 128) return run<128, false, true>(a, stream);
+    if (a.D == 64) return run<64, false, true>(a, stream);
     return -2;
   }
-  if (a.D == 128) return run<128, false>(a, stream);
-  if (a.D == 64) return run<64, false>(a, stream);
+  if (a.fp8) {
+    if (a.D == 128) return run<128, true, false>(a, stream);
+    return -2;
+  }
+  if (a.D == 128) return run<128, false, false>(a, stream);
+  if (a.D == 64) return run<64, false, false>(a, stream);
   return -2;
 }
 

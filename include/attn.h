@@ -195,6 +195,53 @@ ATTN_API int attn_decode_paged_multi(const void* q, const void* k_pages, const v
                                      void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_prefill_paged -- chunked prefill over a paged KV cache: the last Lq
+ * cached tokens of every sequence are the queries, and query token i sees the
+ * cached tokens 0 .. seq_lens[b] - Lq + i (the causal mask aligned at the
+ * bottom-right corner, as in attn_fwd; with window > 0 only the last window
+ * of them).  Their K/V must already be in the pool (attn_kv_append).  The
+ * same tiled kernel as attn_fwd, its K/V tiles gathered page by page through
+ * the block table (PagedAttention section of the zeeklog page).
+ *
+ *   q           [B, Hq, Lq, D] bf16
+ *   k_pages     [num_pages, page_size, Hkv, D] bf16, shared pool (num_pages >= 1)
+ *   v_pages     [num_pages, page_size, Hkv, D] bf16
+ *   block_table [B, max_pages_per_seq] int32 (entries past a sequence's length
+ *               are not read)
+ *   seq_lens    [B] int32 (device): cached tokens, the Lq new ones included;
+ *               clamped to max_pages_per_seq * page_size
+ *   o           [B, Hq, Lq, D] bf16 (written); lse [B, Hq, Lq] fp32 (written;
+ *               may be NULL)
+ *
+ * Rows without any visible token get O = 0, LSE = -inf; cache slots past
+ * seq_lens[b] are never used, whatever they hold.  Page ids are read through
+ * the pool's tensor map: an id outside the pool reads zeros, never faults.
+ * Supported: bf16, D in {64, 128}, page_size == 16, Hq % Hkv == 0.
+ */
+ATTN_API int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int* block_table, const int* seq_lens, void* o, float* lse,
+                                int B, int Hq, int Hkv, int Lq, int D, int page_size, int num_pages,
+                                int max_pages_per_seq, float scale, int window, attn_stream_t stream);
+
+/*
+ * attn_kv_append -- write the K/V of each sequence's L_new newest tokens into
+ * their slots of the page pools: token t of sequence b goes to position
+ * seq_lens[b] - L_new + t (seq_lens counts the new tokens), i.e. page
+ * block_table[b][pos / page_size], slot pos % page_size.  Positions below 0
+ * are skipped.
+ *
+ *   k_new, v_new  [B, Hkv, L_new, D] bf16 (read)
+ *   k_pages, v_pages, block_table, seq_lens as attn_prefill_paged (pools written)
+ *
+ * Every page id is checked before the write: one outside [0, num_pages) is
+ * skipped and reported as ATTN_ERR_BOUNDS by attn_last_device_error().
+ * Supported: D a multiple of 8, page_size == 16.
+ */
+ATTN_API int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                            const int* block_table, const int* seq_lens, int B, int Hkv, int L_new, int D,
+                            int page_size, int num_pages, int max_pages_per_seq, attn_stream_t stream);
+
+/*
  * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot
  * allocate device memory at the call site (no counterpart in the pages this
  * library follows).

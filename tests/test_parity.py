@@ -257,6 +257,101 @@ def test_decode_multi_of_one_token_is_decode(lib):
     assert torch.equal(o1, o2[:, :, 0]) and torch.equal(l1, l2[:, :, 0])
 
 
+# ------------------------------------------- chunked prefill over pages, KV append
+def _paged_case(lens, Hq, Hkv, D, seed, nan_tail=False):
+    shape = DecodeShape("paged", B=len(lens), Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=1)
+    kv = decode_inputs(shape, seed, seq_lens=lens, extra_pages=3)
+    if nan_tail:
+        for b, n in enumerate(lens):
+            npg = (n + 15) // 16
+            if npg and n % 16:
+                last = int(kv.block_table[b, npg - 1])
+                kv.k_pages[last, n % 16:] = float("nan")
+                kv.v_pages[last, n % 16:] = float("nan")
+    return shape, kv
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,Lq,D,window,nan_tail", [
+    ([500, 200, 1000], 8, 2, 200, 128, 0, False),     # GQA, chunk after a cached prefix
+    ([130, 77], 4, 4, 130, 64, 0, False),              # MHA, one cache shorter than the chunk
+    ([700, 300], 6, 2, 256, 128, 100, True),           # group of 3, sliding window, NaN tail slots
+    ([129, 16, 1], 32, 8, 17, 128, 0, True),
+])
+def test_prefill_paged(lib, lens, Hq, Hkv, Lq, D, window, nan_tail):
+    shape, kv = _paged_case(lens, Hq, Hkv, D, 90 + Lq, nan_tail)
+    q = decode_queries(shape, Lq, 91 + Lq)
+    d = {n: getattr(kv, n).cuda() for n in ("k_pages", "v_pages", "block_table", "seq_lens")}
+    o, lse = lib.attn_prefill_paged(q.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                    shape.scale, window)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    o_ref, l_ref = oracle.paged_decode(q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale,
+                                       window=window)
+    assert torch.isfinite(o.float()).all()
+    _check(o, o_ref, lse, l_ref, what=f"paged prefill {lens} Lq={Lq} W={window}")
+
+
+def test_prefill_paged_equals_contiguous_prefill(lib):
+    """Sequences of equal length whose whole cache is the chunk: the paged
+    kernel reads the same K/V blocks as attn_fwd on the contiguous tensors and
+    must give identical bits."""
+    B, Hq, Hkv, L, D = 2, 8, 2, 384, 128
+    shape = DecodeShape("eq", B=B, Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=1)
+    kv = decode_inputs(shape, 95, seq_lens=[L] * B)
+    q = decode_queries(shape, L, 96)
+    k = torch.stack([torch.from_numpy(oracle.gather_pages(kv.k_pages, kv.block_table[b], L, 16)).to(torch.bfloat16)
+                     .permute(1, 0, 2) for b in range(B)])
+    v = torch.stack([torch.from_numpy(oracle.gather_pages(kv.v_pages, kv.block_table[b], L, 16)).to(torch.bfloat16)
+                     .permute(1, 0, 2) for b in range(B)])
+    d = {n: getattr(kv, n).cuda() for n in ("k_pages", "v_pages", "block_table", "seq_lens")}
+    o1, l1 = lib.attn_prefill_paged(q.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                    shape.scale)
+    o2, l2 = lib.attn_fwd(q.cuda(), k.contiguous().cuda(), v.contiguous().cuda(), shape.scale, True, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_kv_append_then_prefill(lib):
+    """Append a chunk's K/V into the pages (exactly the oracle's scatter), then
+    attend the chunk over the whole cache."""
+    lens, Ln = [300, 40, 17], 40
+    shape, kv = _paged_case(lens, 8, 2, 128, 97)
+    g = torch.Generator().manual_seed(98)
+    k_new = torch.randn(3, 2, Ln, 128, generator=g).to(torch.bfloat16)
+    v_new = torch.randn(3, 2, Ln, 128, generator=g).to(torch.bfloat16)
+    d = {n: getattr(kv, n).cuda() for n in ("k_pages", "v_pages", "block_table", "seq_lens")}
+    lib.attn_kv_append(k_new.cuda(), v_new.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"])
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    kp_ref, vp_ref = oracle.kv_append(kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, k_new, v_new)
+    assert np.array_equal(d["k_pages"].double().cpu().numpy(), kp_ref)
+    assert np.array_equal(d["v_pages"].double().cpu().numpy(), vp_ref)
+    q = decode_queries(shape, Ln, 99)
+    o, lse = lib.attn_prefill_paged(q.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                    shape.scale)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.paged_decode(q, kp_ref, vp_ref, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, o_ref, lse, l_ref, what="append + paged prefill")
+
+
+def test_kv_append_rejects_bad_page_ids(lib):
+    shape, kv = _paged_case([40, 20], 4, 2, 128, 100)
+    kv.block_table[1, 0] = kv.num_pages + 3
+    k_new = torch.zeros(2, 2, 8, 128, dtype=torch.bfloat16)
+    d = {n: getattr(kv, n).cuda() for n in ("k_pages", "v_pages", "block_table", "seq_lens")}
+    before = d["k_pages"].clone()
+    lib.attn_kv_append(k_new.cuda(), k_new.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"])
+    assert lib.attn_last_device_error() == lib.ATTN_ERR_BOUNDS
+    # sequence 0 was written; of sequence 1 (positions 12..19) only the
+    # tokens on its good page (16..19) were, the ones on the bad page skipped
+    kp_ref, vp_ref = oracle.kv_append(kv.k_pages, kv.v_pages, kv.block_table[:1], kv.seq_lens[:1], k_new[:1],
+                                      k_new[:1])
+    kp_ref, _ = oracle.kv_append(kp_ref, vp_ref, kv.block_table[1:], kv.seq_lens[1:], k_new[1:, :, 4:],
+                                 k_new[1:, :, 4:])
+    assert np.array_equal(d["k_pages"].double().cpu().numpy(), kp_ref)
+    assert not torch.equal(before, d["k_pages"])
+
+
 def test_decode_invariant_to_page_permutation(lib):
     shape = DecodeShape("perm", B=4, Hq=32, Hkv=1, D=128, len_lo=100, len_hi=900)
     kv = decode_inputs(shape, 5)
