@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PROFILED_TRAFFIC = {
     "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "cf6866cd14575b31",
                 "bytes": 307_631_360 + 97_784_576, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
-    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "498976c04c88a208",
-               "bytes": 147_962_112 + 4_209_664, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
+    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "f9baebc778a8a9a4",
+               "bytes": 147_916_544 + 4_712_960, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
 }
 
 
@@ -466,7 +466,50 @@ def side_workloads(attn, dev, peaks, world):
         del fn
         torch.cuda.empty_cache()
     out.update(multi_token_decode(attn, dev, peaks, world))
+    out.update(paged_chunk_prefill(attn, dev, peaks, world))
     return out
+
+
+def paged_chunk_prefill(attn, dev, peaks, world, B=4, Hq=32, Hkv=8, D=128, cached=3072, chunk=1024):
+    """Chunked prefill over a paged cache (attn_prefill_paged): each of B
+    sequences holds `cached` tokens plus a `chunk` of new ones, 16-token pages
+    in a permuted pool; the chunk attends causally to all of them.  Also the
+    KV append of the chunk (attn_kv_append).  Median of 5 after 2 warm-ups."""
+    import torch
+    from workloads import DecodeShape
+    shape = DecodeShape("paged_chunk", B=B, Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=1)
+    L = cached + chunk
+    kv = decode_inputs(shape, seed_of(1) + 200, seq_lens=[L] * B)
+    q = decode_queries(shape, chunk, seed_of(1) + 201).to(dev)
+    kp, vp, bt, sl = kv.k_pages.to(dev), kv.v_pages.to(dev), kv.block_table.to(dev), kv.seq_lens.to(dev)
+    g = torch.Generator().manual_seed(seed_of(1) + 202)
+    k_new = torch.randn(B, Hkv, chunk, D, generator=g).to(torch.bfloat16).to(dev)
+    v_new = torch.randn(B, Hkv, chunk, D, generator=g).to(torch.bfloat16).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return max_over_ranks(statistics.median(ts), world, dev)
+
+    ms = timed(lambda: attn.attn_prefill_paged(q, kp, vp, bt, sl, shape.scale, o=o, lse=lse))
+    flops = 4.0 * D * Hq * B * (chunk * cached + chunk * (chunk + 1) / 2)
+    tf = flops / (ms / 1e3) / 1e12
+    ms_app = timed(lambda: attn.attn_kv_append(k_new, v_new, kp, vp, bt, sl))
+    app_bytes = 2 * 2 * B * Hkv * chunk * D * 2  # K and V, read and written
+    return {f"paged_chunk_prefill_B{B}_H{Hq}_G{Hq // Hkv}_cached{cached}_chunk{chunk}_D{D}": {
+        "TFLOP/s": round(tf, 1), "ms": round(ms, 3), "frac": round(tf / peaks["bf16_tflops"], 4),
+        "kv_append_GB/s": round(app_bytes / (ms_app / 1e3) / 1e9, 1), "kv_append_us": round(ms_app * 1e3, 2)}}
 
 
 def multi_token_decode(attn, dev, peaks, world, q_len: int = 4):
