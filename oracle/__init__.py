@@ -27,6 +27,7 @@ formula against allocated bytes.  No function here is "parity unpinned".
 """
 from .sdpa import (  # noqa: F401
     attention,
+    attention_backward,
     attention_fp8,
     dequantize_e4m3,
     gather_pages,

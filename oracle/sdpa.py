@@ -140,6 +140,53 @@ def dequantize_e4m3(x8, s: float) -> np.ndarray:
     return _f64(x8) * float(s)
 
 
+def attention_backward(q, k, v, o, do, lse, scale: float, causal: bool = False, window: int = 0):
+    """Gradients of O = softmax(scale * Q K^T + mask) V with respect to Q, K
+    and V, in float64, from the forward's O and per-row LSE.
+
+    Follows the recomputation of the tqpw.cn article §4.1 (the backward pass
+    recomputes the attention weights instead of storing them; p5 §一 notes the
+    stored score matrix as the cost being avoided): P = exp(scale * Q K^T -
+    LSE) row by row (masked entries 0), then with Dvec = rowsum(dO * O)
+
+        dV = P^T dO,   dP = dO V^T,   dS = P * (dP - Dvec),
+        dQ = scale * dS K,   dK = scale * dS^T Q.
+
+    GQA/MQA: the K/V gradients of a K/V head sum over the query heads of its
+    group.  Layout [B, H, L, D] as ``attention``.  Returns (dQ, dK, dV)."""
+    q, k, v, o, do = (_f64(x) for x in (q, k, v, o, do))
+    lse = _f64(lse)
+    B, Hq, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    group = Hq // Hkv
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    lo_all, hi_all = _row_ranges(Lq, Lk, causal, window, np.arange(Lq))
+    chunk = max(1, _MAX_SCORE_ELEMS // max(Lk, 1))
+    cols = np.arange(Lk)[None, :]
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // group
+            for r0 in range(0, Lq, chunk):
+                r1 = min(Lq, r0 + chunk)
+                lo, hi = lo_all[r0:r1], hi_all[r0:r1]
+                s = scale * (q[b, h, r0:r1] @ k[b, kvh].T)
+                masked = (cols < lo[:, None]) | (cols >= hi[:, None])
+                li = lse[b, h, r0:r1]
+                p_ = np.zeros_like(s)
+                live = np.isfinite(li)
+                p_[live] = np.exp(s[live] - li[live][:, None])
+                p_[masked] = 0.0
+                dvec = (do[b, h, r0:r1] * o[b, h, r0:r1]).sum(axis=1)
+                dv[b, kvh] += p_.T @ do[b, h, r0:r1]
+                dp = do[b, h, r0:r1] @ v[b, kvh].T
+                ds = p_ * (dp - dvec[:, None])
+                dq[b, h, r0:r1] = scale * (ds @ k[b, kvh])
+                dk[b, kvh] += scale * (ds.T @ q[b, h, r0:r1])
+    return dq, dk, dv
+
+
 def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale: float,
                   causal: bool = False, window: int = 0, **kw):
     """Attention on e4m3 inputs: the plain definition applied to the exact

@@ -408,6 +408,93 @@ def test_paged_window_equals_contiguous_window():
         np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------------------ backward
+def _autograd_grads(q, k, v, do, scale, causal, window):
+    """Gradients by float64 autograd of a separately written forward (masked
+    softmax of the scores, GQA by repeating K/V heads)."""
+    qt, kt, vt = (torch.tensor(np.asarray(x, dtype=np.float64), requires_grad=True) for x in (q, k, v))
+    B, Hq, Lq, D = qt.shape
+    Hkv, Lk = kt.shape[1], kt.shape[2]
+    kr = kt.repeat_interleave(Hq // Hkv, dim=1)
+    vr = vt.repeat_interleave(Hq // Hkv, dim=1)
+    s = scale * qt @ kr.transpose(-1, -2)
+    i = torch.arange(Lq)[:, None] + (Lk - Lq)
+    j = torch.arange(Lk)[None, :]
+    allowed = torch.ones(Lq, Lk, dtype=torch.bool)
+    if causal:
+        allowed &= j <= i
+        if window > 0:
+            allowed &= j > i - window
+    s = s.masked_fill(~allowed, float("-inf"))
+    out = torch.softmax(s, dim=-1) @ vr
+    out.backward(torch.tensor(np.asarray(do, dtype=np.float64)))
+    return out.detach().numpy(), qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,window", [
+    (1, 2, 2, 5, 5, 4, False, 0),
+    (2, 4, 2, 9, 9, 8, True, 0),
+    (1, 6, 2, 7, 11, 4, True, 0),      # Lq < Lk, bottom-right causal
+    (1, 4, 1, 12, 12, 8, True, 3),     # MQA, sliding window
+])
+def test_attention_backward_equals_autograd(B, Hq, Hkv, Lq, Lk, D, causal, window):
+    g = torch.Generator().manual_seed(21)
+    q = torch.randn(B, Hq, Lq, D, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, Lk, D, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, Lk, D, generator=g, dtype=torch.float64)
+    do = torch.randn(B, Hq, Lq, D, generator=g, dtype=torch.float64)
+    o, lse = oracle.attention(q, k, v, 0.4, causal, window)
+    dq, dk, dv = oracle.attention_backward(q, k, v, o, do, lse, 0.4, causal, window)
+    o_ref, dq_ref, dk_ref, dv_ref = _autograd_grads(q, k, v, do, 0.4, causal, window)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dq, dq_ref, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, dk_ref, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, dv_ref, rtol=0, atol=1e-11)
+
+
+def test_attention_backward_finite_differences():
+    """Central differences of L = sum(O * dO) against the analytic gradients
+    for a few entries of each input."""
+    g = torch.Generator().manual_seed(22)
+    q = torch.randn(1, 2, 6, 4, generator=g, dtype=torch.float64).numpy()
+    k = torch.randn(1, 1, 6, 4, generator=g, dtype=torch.float64).numpy()
+    v = torch.randn(1, 1, 6, 4, generator=g, dtype=torch.float64).numpy()
+    do = torch.randn(1, 2, 6, 4, generator=g, dtype=torch.float64).numpy()
+    o, lse = oracle.attention(q, k, v, 0.5, True, 0)
+    dq, dk, dv = oracle.attention_backward(q, k, v, o, do, lse, 0.5, True, 0)
+
+    def loss(q_, k_, v_):
+        return float((oracle.attention(q_, k_, v_, 0.5, True, 0)[0] * do).sum())
+
+    eps = 1e-6
+    for arr, grad, idx in ((q, dq, (0, 1, 3, 2)), (k, dk, (0, 0, 2, 1)), (v, dv, (0, 0, 4, 3)), (k, dk, (0, 0, 0, 0))):
+        plus, minus = arr.copy(), arr.copy()
+        plus[idx] += eps
+        minus[idx] -= eps
+        args_p = [plus if a is arr else a for a in (q, k, v)]
+        args_m = [minus if a is arr else a for a in (q, k, v)]
+        fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert abs(fd - grad[idx]) < 1e-7, (idx, fd, grad[idx])
+
+
+def test_attention_backward_gqa_sums_over_the_group():
+    """The K/V gradients of a GQA head equal the MHA gradients of the
+    repeat_kv-duplicated heads summed over each group."""
+    g = torch.Generator().manual_seed(23)
+    q = torch.randn(1, 4, 8, 4, generator=g, dtype=torch.float64).numpy()
+    k = torch.randn(1, 2, 8, 4, generator=g, dtype=torch.float64).numpy()
+    v = torch.randn(1, 2, 8, 4, generator=g, dtype=torch.float64).numpy()
+    do = torch.randn(1, 4, 8, 4, generator=g, dtype=torch.float64).numpy()
+    o, lse = oracle.attention(q, k, v, 0.5, True, 0)
+    dq, dk, dv = oracle.attention_backward(q, k, v, o, do, lse, 0.5, True, 0)
+    kr, vr = oracle.repeat_kv(k, 2), oracle.repeat_kv(v, 2)
+    o2, lse2 = oracle.attention(q, kr, vr, 0.5, True, 0)
+    dq2, dk2, dv2 = oracle.attention_backward(q, kr, vr, o2, do, lse2, 0.5, True, 0)
+    np.testing.assert_allclose(dq, dq2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk, dk2.reshape(1, 2, 2, 8, 4).sum(axis=2), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(1, 2, 2, 8, 4).sum(axis=2), rtol=0, atol=1e-13)
+
+
 def test_merge_partials_equals_unsplit():
     """Split the keys into parts, attend each part, merge by LSE: equals
     attention over all keys (float64, to rounding)."""
