@@ -70,6 +70,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_prefill_paged.restype = c_int
     lib.attn_kv_append.argtypes = [c_void_p] * 6 + [c_int] * 7 + [c_void_p]
     lib.attn_kv_append.restype = c_int
+    lib.attn_bwd_workspace_bytes.argtypes = [c_int] * 4
+    lib.attn_bwd_workspace_bytes.restype = c_size_t
+    lib.attn_bwd.argtypes = [c_void_p] * 9 + [c_int] * 6 + [c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]
+    lib.attn_bwd.restype = c_int
     lib.attn_decode_paged_noalloc.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p]
     lib.attn_decode_paged_noalloc.restype = c_int
     lib.attn_last_device_error.argtypes = [c_void_p]
@@ -258,6 +262,30 @@ def attn_kv_append(k_new, v_new, k_pages, v_pages, block_table, seq_lens, stream
                             _stream_handle(stream))
     _check(st, "attn_kv_append")
     return k_pages, v_pages
+
+
+def attn_bwd(q, k, v, o, dout, lse, scale: Optional[float] = None, causal: bool = False, window: int = 0,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of attn_fwd: q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D], o and dout
+    [B,Hq,Lq,D] bf16, lse [B,Hq,Lq] fp32 (attn_fwd's).  Returns (dq, dk, dv)
+    bf16."""
+    import torch
+    lib = load()
+    B, Hq, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = lib.attn_bwd_workspace_bytes(B, Hq, Lq, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                      B, Hq, Hkv, Lq, Lk, D, float(scale), int(bool(causal)), int(window), _ptr(workspace),
+                      workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,

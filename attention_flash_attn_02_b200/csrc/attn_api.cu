@@ -195,6 +195,34 @@ ATTN_API int attn_kv_append(const void* k_new, const void* v_new, void* k_pages,
                           max_pages_per_seq, static_cast<cudaStream_t>(stream));
 }
 
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Lq, int D) {
+  if (B <= 0 || Hq <= 0 || Lq <= 0 || D <= 0) return 0;
+  return backward_workspace_bytes(B, Hq, Lq, D);
+}
+
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                      float scale, int causal, int window, void* workspace, size_t workspace_bytes,
+                      attn_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || D <= 0) return ATTN_ERR_INVALID;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
+  if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;
+  if (window > 0 && !causal) return ATTN_ERR_INVALID;
+  if (causal && Lq > Lk) return ATTN_ERR_INVALID;
+  if (B == 0 || Lq == 0) return ATTN_OK;
+  const void* ptrs[] = {q, o, dout, dq, workspace};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return ATTN_ERR_INVALID;
+  if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID;
+  if (Lk > 0 && (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv)))
+    return ATTN_ERR_INVALID;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (workspace_bytes < attn_bwd_workspace_bytes(B, Hq, Lq, D)) return ATTN_ERR_INVALID;
+  BackwardArgs a{q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Lq, Lk, D, scale, causal ? 1 : 0,
+                 window > 0 ? window : 0, workspace};
+  return launch_backward(a, static_cast<cudaStream_t>(stream));
+}
+
 ATTN_API int attn_last_device_error(attn_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
   int* p = device_status_word();

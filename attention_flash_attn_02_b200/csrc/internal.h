@@ -55,6 +55,27 @@ int fail_cuda(const char* where, cudaError_t err);
 
 // Launchers: return a status code of include/attn.h.
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+
+struct BackwardArgs {
+  const void* q;     // [B, Hq, Lq, D] bf16
+  const void* k;     // [B, Hkv, Lk, D]
+  const void* v;
+  const void* o;     // forward output [B, Hq, Lq, D]
+  const void* dout;  // dO
+  const float* lse;  // forward LSE [B, Hq, Lq] (natural log)
+  void* dq;          // [B, Hq, Lq, D] bf16
+  void* dk;          // [B, Hkv, Lk, D]
+  void* dv;
+  int B, Hq, Hkv, Lq, Lk, D;
+  float scale;
+  int causal, window;
+  void* workspace;   // backward_workspace_bytes(...)
+};
+int launch_backward(const BackwardArgs& a, cudaStream_t stream);
+// dQ accumulator [B*Hq*Lq][D] fp32, then LSE (log2) and Dvec [B*Hq*Lq] fp32.
+inline size_t backward_workspace_bytes(int B, int Hq, int Lq, int D) {
+  return (size_t)B * Hq * Lq * (size_t)(D + 2) * 4;
+}
 // New tokens' K/V into their slots of the page pools (KV append).
 int launch_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages, const int* block_table,
                      const int* seq_lens, int B, int Hkv, int L_new, int D, int num_pages, int max_pages,

@@ -122,6 +122,37 @@ ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
                           attn_stream_t stream);
 
 /*
+ * attn_bwd_workspace_bytes -- scratch attn_bwd needs: an fp32 dQ accumulator
+ * of B * Hq * Lq * D floats plus two floats per query row (LSE in log2 units
+ * and rowsum(dO * O)): B * Hq * Lq * (D + 2) * 4 bytes.  0 for empty shapes.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Lq, int D);
+
+/*
+ * attn_bwd -- gradients of attn_fwd (no counterpart call in the pages, which
+ * describe the backward only as recomputing the attention weights from
+ * stored statistics instead of keeping them: tqpw.cn article §4.1).
+ *
+ *   q, k, v, o   as attn_fwd (o = its output), bf16
+ *   dout         [B, Hq, Lq, D] bf16: gradient of the loss with respect to O
+ *   lse          [B, Hq, Lq] fp32: attn_fwd's LSE (natural log)
+ *   dq           [B, Hq, Lq, D] bf16 (written)
+ *   dk, dv       [B, Hkv, Lk, D] bf16 (written; each K/V head sums its group)
+ *   workspace    at least attn_bwd_workspace_bytes(B, Hq, Lq, D) bytes;
+ *                contents on entry do not matter
+ *   scale, causal, window as attn_fwd (same mask, same alignment)
+ *
+ * P = exp(scale * q k^T - lse) is recomputed, rounded to bf16 for the
+ * dV = P^T dO product, and dS = P * (dP - rowsum(dO * O)) to bf16 for the
+ * dK and dQ products; accumulation in fp32.  Supported: bf16, D in {64, 128}.
+ */
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv,
+                      int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                      float scale, int causal, int window,
+                      void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_workspace_bytes -- size of the scratch buffer attn_decode_paged
  * needs for these sizes: per query head of every sequence, up to
  * S = ceil(max_pages_per_seq / 32) + 1 partial results of D + 1 floats

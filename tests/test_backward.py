@@ -1,0 +1,77 @@
+"""GPU parity of attn_bwd (dQ, dK, dV) against the float64 oracle's
+gradients of the exact definition.
+
+The kernel is fed the GPU forward's own O (bf16) and LSE, as a training step
+would; the oracle differentiates the exact forward.  Tolerance: the products
+round P and dS to bf16 (relative 2^-9) and the outputs are bf16, so each
+gradient is compared relative to its own scale: max |err| <= 2e-2 * max |ref|
+and mean |err| <= 4e-3 * mean |ref| (about ten and two bf16 half-ulps).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import PrefillShape, prefill_inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL, MEAN_REL = 2e-2, 4e-3
+
+
+def _grad_check(name, got, ref):
+    got = got.float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    scale_max, scale_mean = np.abs(ref).max(), np.abs(ref).mean()
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    assert err.max() <= MAX_REL * scale_max + 1e-6, f"{name}: max {err.max():.3e} vs {MAX_REL * scale_max:.3e}"
+    assert err.mean() <= MEAN_REL * scale_mean + 1e-7, f"{name}: mean {err.mean():.3e} vs {MEAN_REL * scale_mean:.3e}"
+    return err.max() / scale_max, err.mean() / scale_mean
+
+
+def _case(lib, B, Hq, Hkv, Lq, Lk, D, causal, window, seed):
+    shape = PrefillShape("bwd", B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, D=D, causal=causal, window=window)
+    q, k, v = prefill_inputs(shape, seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    do = torch.randn(B, Hq, Lq, D, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = lib.attn_fwd(qd, kd, vd, shape.scale, causal, window)
+    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, dod, lse, shape.scale, causal, window)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    o_ref, l_ref = oracle.attention(q, k, v, shape.scale, causal, window)
+    dq_r, dk_r, dv_r = oracle.attention_backward(q, k, v, o_ref, do, l_ref, shape.scale, causal, window)
+    return [_grad_check(n, a, r) for n, a, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r))]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,window", [
+    (1, 2, 2, 128, 128, 64, False, 0),      # one tile each way
+    (2, 4, 2, 300, 300, 128, True, 0),      # ragged tails, GQA
+    (1, 8, 2, 512, 512, 128, True, 0),      # group of 4
+    (1, 4, 1, 130, 400, 64, True, 0),       # MQA, Lq < Lk (bottom-right causal)
+    (1, 4, 2, 700, 700, 128, True, 200),    # sliding window
+    (1, 6, 2, 257, 257, 128, False, 0),     # group of 3, non-causal
+])
+def test_backward_parity(lib, B, Hq, Hkv, Lq, Lk, D, causal, window):
+    _case(lib, B, Hq, Hkv, Lq, Lk, D, causal, window, 500 + Lq + Hq)
+
+
+def test_backward_gqa_causal_1k(lib):
+    """The GQA causal shape of the prefill workload at 1024 tokens (group 4,
+    D = 128): eight 128-key tiles per head, causal skipping on both sides."""
+    _case(lib, 1, 8, 2, 1024, 1024, 128, True, 0, 601)
+
+
+def test_backward_repeat_is_bitwise_stable(lib):
+    """dK and dV are accumulated in TMEM by one CTA each and come out
+    bit-identical on a second run; dQ is summed with fp32 reductions in
+    arbitrary order and only agrees to rounding."""
+    shape = PrefillShape("bwd", B=1, Hq=4, Hkv=2, Lq=384, Lk=384, D=128, causal=True)
+    q, k, v = [t.cuda() for t in prefill_inputs(shape, 602)]
+    do = torch.randn(1, 4, 384, 128, generator=torch.Generator().manual_seed(603)).to(torch.bfloat16).cuda()
+    o, lse = lib.attn_fwd(q, k, v, shape.scale, True, 0)
+    g1 = lib.attn_bwd(q, k, v, o, do, lse, shape.scale, True, 0)
+    g2 = lib.attn_bwd(q, k, v, o, do, lse, shape.scale, True, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+    assert torch.allclose(g1[0].float(), g2[0].float(), atol=1e-2, rtol=1e-2)
