@@ -162,6 +162,10 @@ def attn_decode_workspace_bytes(B: int, Hq: int, max_pages_per_seq: int, D: int)
     return int(load().attn_decode_workspace_bytes(B, Hq, max_pages_per_seq, D))
 
 
+def attn_bwd_workspace_bytes(B: int, Hq: int, Lq: int, D: int) -> int:
+    return int(load().attn_bwd_workspace_bytes(B, Hq, Lq, D))
+
+
 def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,
                       o=None, lse=None, workspace=None, stream=None):
     """Single-token paged decode.  q [B,Hq,D] bf16; pools [P,16,Hkv,D] bf16;
@@ -278,7 +282,7 @@ def attn_bwd(q, k, v, o, dout, lse, scale: Optional[float] = None, causal: bool 
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    need = lib.attn_bwd_workspace_bytes(B, Hq, Lq, D)
+    need = attn_bwd_workspace_bytes(B, Hq, Lq, D)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),

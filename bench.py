@@ -467,7 +467,41 @@ def side_workloads(attn, dev, peaks, world):
         torch.cuda.empty_cache()
     out.update(multi_token_decode(attn, dev, peaks, world))
     out.update(paged_chunk_prefill(attn, dev, peaks, world))
+    out.update(backward_pass(attn, dev, peaks, world))
     return out
+
+
+def backward_pass(attn, dev, peaks, world):
+    """attn_bwd on the GQA causal prefill workload (its own forward's O and
+    LSE): 5 products of the visible (query, key) pairs against the forward's
+    2, i.e. 2.5x the forward's FLOPs.  Median of 5 after 2 warm-ups; the
+    inputs (201 MB) and the dQ accumulator (272 MB) exceed L2."""
+    import torch
+    shape = PREFILL
+    q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(1))]
+    g = torch.Generator().manual_seed(seed_of(1) + 300)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    o, lse = attn.attn_fwd(q, k, v, shape.scale, shape.causal, shape.window)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.attn_bwd_workspace_bytes(shape.B, shape.Hq, shape.Lq, shape.D), dtype=torch.uint8,
+                     device=dev)
+    fn = lambda: attn.attn_bwd(q, k, v, o, do, lse, shape.scale, shape.causal, shape.window,  # noqa: E731
+                               dq=dq, dk=dk, dv=dv, workspace=ws)
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = max_over_ranks(statistics.median(ts), world, dev)
+    tf = 2.5 * prefill_flops(shape) / (ms / 1e3) / 1e12
+    return {f"backward_{shape.name}": {"TFLOP/s": round(tf, 1), "ms": round(ms, 3),
+                                       "frac": round(tf / peaks["bf16_tflops"], 4)}}
 
 
 def paged_chunk_prefill(attn, dev, peaks, world, B=4, Hq=32, Hkv=8, D=128, cached=3072, chunk=1024):

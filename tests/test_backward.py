@@ -75,3 +75,25 @@ def test_backward_repeat_is_bitwise_stable(lib):
     torch.cuda.synchronize()
     assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
     assert torch.allclose(g1[0].float(), g2[0].float(), atol=1e-2, rtol=1e-2)
+
+
+def test_backward_full_size_first_group(lib):
+    """The GQA causal prefill workload (B4 Hq32 Hkv8 L4096 D128) end to end on
+    the GPU; the oracle checks batch 0's first K/V group (query heads 0-3 and
+    K/V head 0), whose gradients depend on nothing else."""
+    from workloads import GQA_CAUSAL, seed_of
+    shape = GQA_CAUSAL
+    q, k, v = prefill_inputs(shape, seed_of(1))
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(seed_of(1) + 300)).to(torch.bfloat16)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = lib.attn_fwd(qd, kd, vd, shape.scale, True, 0)
+    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, dod, lse, shape.scale, True, 0)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    g = shape.Hq // shape.Hkv
+    qs, ks, vs, dos = q[:1, :g], k[:1, :1], v[:1, :1], do[:1, :g]
+    o_ref, l_ref = oracle.attention(qs, ks, vs, shape.scale, True, 0)
+    dq_r, dk_r, dv_r = oracle.attention_backward(qs, ks, vs, o_ref, dos, l_ref, shape.scale, True, 0)
+    _grad_check("dq", dq[:1, :g], dq_r)
+    _grad_check("dk", dk[:1, :1], dk_r)
+    _grad_check("dv", dv[:1, :1], dv_r)
