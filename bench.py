@@ -43,8 +43,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sources they were taken on (sha256 prefix of the files); a changed kernel
 # reports null until it is captured again.
 PROFILED_TRAFFIC = {
-    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "cf6866cd14575b31",
-                "bytes": 307_631_360 + 97_784_576, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
+    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "5d4bea9f89ab10b5",
+                "bytes": 312_252_928 + 97_561_600, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
     "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "f9baebc778a8a9a4",
                "bytes": 147_916_544 + 4_712_960, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
 }
