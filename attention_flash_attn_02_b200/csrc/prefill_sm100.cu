@@ -63,9 +63,36 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Of every 8 pairs of exponentials, this many are computed by the FMA-pipe
 // polynomial instead of the MUFU ex2 unit (balances the two pipes).
 #ifndef ATTN_EMU_PAIRS_PER8
-#define ATTN_EMU_PAIRS_PER8 2
+#define ATTN_EMU_PAIRS_PER8 0
 #endif
-constexpr int kEmuPairsPer8 = ATTN_EMU_PAIRS_PER8;
+#ifndef ATTN_EMU_PAIRS_PER8_FP8
+#define ATTN_EMU_PAIRS_PER8_FP8 2
+#endif
+template <bool FP8>
+constexpr int kEmuPairsPer8 = FP8 ? ATTN_EMU_PAIRS_PER8_FP8 : ATTN_EMU_PAIRS_PER8;
+// P handoff in two parts: after the first ATTN_SPLIT_P x 16 keys of the block
+// (0: no split; 2, 4 or 6 of 8) the MMA warp starts O += P V on them while the
+// softmax warps compute the rest.
+#ifndef ATTN_SPLIT_P
+#define ATTN_SPLIT_P 6
+#endif
+constexpr bool kSplitP = ATTN_SPLIT_P != 0;
+#ifndef ATTN_EARLY_Q
+#define ATTN_EARLY_Q 1
+#endif
+constexpr bool kEarlyQ = ATTN_EARLY_Q != 0;
+constexpr int kSplitKeys = ATTN_SPLIT_P * 16;
+static_assert(ATTN_SPLIT_P == 0 || (ATTN_SPLIT_P % 2 == 0 && ATTN_SPLIT_P < 8), "split at 32, 64 or 96 keys");
+// bf16 path: O is normalised by the sum of the bf16-rounded P that the MMA
+// multiplies (1: halves unpacked by shift and mask, added in pairs; 2: each
+// half added by a mixed-precision bf16 + f32 add) or by the exact fp32 row
+// sum (0); 3: as 1, but summed from the packed words after P has been handed
+// to the MMA warp, while the warp waits for its next S.  On rows of a few keys the two sums differ by up to 2^-10, which
+// with the bf16 rounding of O can exceed 1e-2 absolute.  The e4m3 path always
+// uses the rounded sum.
+#ifndef ATTN_ROUNDED_SUM
+#define ATTN_ROUNDED_SUM 1
+#endif
 
 template <int D, bool FP8>
 struct Cfg {
@@ -214,6 +241,7 @@ __device__ __forceinline__ int unit_of(int round, int n_units) {
 struct Smem {
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], p_full[2];
+  uint64_t p_half[2];         // first 64 keys of P stored (128 arrivals)
   uint64_t o_full[2], o_empty[2];
   uint64_t drain;
   uint64_t kv_full[12], kv_empty[12];
@@ -227,6 +255,50 @@ struct Smem {
 };
 
 static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserve");
+
+// One pair of keys of a softmax row: x = s * scale * log2e - m, P = 2^x (MUFU
+// ex2, or for kEmuPairsPer8 of every 8 pairs the FMA-pipe polynomial), packed
+// for the MMA, added to the exact row sum and, with RSUM, to the sum of the
+// rounded values.  e4m3 pairs go two to a 32-bit word.
+template <bool FP8, int RSUM>
+__device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
+                                       uint64_t (&rs2)[4], uint64_t (&rr2)[4], float (&rrs)[8],
+                                       uint32_t (&pk)[kBN / 2]) {
+  const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
+  float p0, p1;
+  if ((q2 & 7) >= 8 - kEmuPairsPer8<FP8>) {
+    f2_split(exp2_poly2(x2), p0, p1);
+  } else {
+    float x0, x1;
+    f2_split(x2, x0, x1);
+    p0 = ex2_approx(x0);
+    p1 = ex2_approx(x1);
+  }
+  rs2[q2 & 3] = add2(rs2[q2 & 3], f2(p0, p1));
+  if (FP8) {
+    const uint16_t e = pack_e4m3x2(p0, p1);
+    if (q2 & 1) pk[q2 >> 1] |= (uint32_t)e << 16;
+    else pk[q2 >> 1] = e;
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(e));
+    float h0, h1;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(h0), "=f"(h1)
+        : "r"(h));
+    rr2[q2 & 3] = add2(rr2[q2 & 3], f2(h0, h1));
+  } else {
+    const uint32_t b = pack_bf16x2(p0, p1);
+    pk[q2] = b;
+    if (RSUM == 1) {
+      rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
+    } else if (RSUM == 2) {
+      asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+          "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+          : "+f"(rrs[2 * (q2 & 3)]), "+f"(rrs[2 * (q2 & 3) + 1])
+          : "r"(b));
+    }
+  }
+}
 
 template <int D, bool FP8, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -250,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_empty[t], 1);
       mbar_init(&sm.s_full[t], 1);
       mbar_init(&sm.p_full[t], 128);
+      mbar_init(&sm.p_half[t], 128);
       mbar_init(&sm.o_full[t], 1);
       mbar_init(&sm.o_empty[t], 128);
       mbar_init(&sm.st_full[t], 128);
@@ -446,10 +519,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O_t (+)= P_t V: P from TMEM (over S_t), V MN-major, 128-byte column
       // groups BOX_BYTES apart, k-step kk = MMA_K keys of 128-byte rows.
-      auto issue_pv = [&](int t, uint32_t v_stage_addr, bool acc) {
+      // k-steps [k_lo, k_hi) of the block's PV_KSTEPS.
+      auto issue_pv = [&](int t, uint32_t v_stage_addr, bool acc, int k_lo, int k_hi) {
         const uint64_t b0 = sw128_desc(v_stage_addr, C::BOX_BYTES, 1024);
 #pragma unroll
-        for (int kk = 0; kk < C::PV_KSTEPS; ++kk) {
+        for (int kk = k_lo; kk < k_hi; ++kk) {
           const uint32_t a = tS(t) + kk * (C::MMA_K * C::EL / 4);
           const uint32_t off = (kk * C::MMA_K * 128) >> 4;
           if (FP8)
@@ -469,10 +543,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         ++seq;
+        // q_empty[t] is committed after the unit's last S of tile t (its last
+        // reader of Q_t), so that the next unit's Q and first K/V tiles load
+        // while this unit's last softmax and P V run.
         issue_s(0, kv_addr0 + sk * C::TILE_BYTES);
         tc_commit(&sm.s_full[0]);
+        if (kEarlyQ && w.nb == 1) tc_commit(&sm.q_empty[0]);
         issue_s(1, kv_addr0 + sk * C::TILE_BYTES);
         tc_commit(&sm.s_full[1]);
+        if (kEarlyQ && w.nb == 1) tc_commit(&sm.q_empty[1]);
         tc_commit(&sm.kv_empty[sk]);
         for (int j = 0; j < w.nb && ok; ++j) {
           const uint32_t sv = seq % C::NS;
@@ -501,14 +580,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool has_next = j + 1 < w.nb;
           const uint32_t skn = seq % C::NS;
           for (int t = 0; t < 2 && ok; ++t) {
-            ok = mbar_wait(&sm.p_full[t], pcnt & 1, g);
+            ok = mbar_wait(kSplitP ? &sm.p_half[t] : &sm.p_full[t], pcnt & 1, g);
             if (!ok) break;
             if (j == 0 && nunit > 0) {
               ok = mbar_wait(&sm.o_empty[t], (nunit - 1) & 1, g);
               if (!ok) break;
             }
             tc_fence_after();
-            issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0);
+            if (kSplitP) {
+              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, kSplitKeys / C::MMA_K);
+              ok = mbar_wait(&sm.p_full[t], pcnt & 1, g);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS);
+            } else {
+              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, C::PV_KSTEPS);
+            }
             if (!has_next) tc_commit(&sm.o_full[t]);
             if (has_next) {
               if (t == 0) {
@@ -518,6 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               issue_s(t, kv_addr0 + skn * C::TILE_BYTES);
               tc_commit(&sm.s_full[t]);
+              if (kEarlyQ && j + 2 == w.nb) tc_commit(&sm.q_empty[t]);
             }
           }
           if (!ok) break;
@@ -529,8 +617,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit(&sm.q_empty[0]);
-        tc_commit(&sm.q_empty[1]);
+        if (!kEarlyQ) {
+          tc_commit(&sm.q_empty[0]);
+          tc_commit(&sm.q_empty[1]);
+        }
         ++nunit;
       }
       // Drain: all issued MMAs complete before TMEM is released.
@@ -548,6 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + (t == 0 ? C::TM_S0 : C::TM_S1) + lane_off;
     const uint32_t tO = tmem + (t == 0 ? C::TM_O0 : C::TM_O1) + lane_off;
     const float sl2 = p.scale_log2;
+    constexpr int kRsum = FP8 ? 1 : ATTN_ROUNDED_SUM;
+    constexpr int kRsumInline = kRsum == 3 ? 0 : kRsum;
     uint32_t scnt = 0, nunit = 0;
     bool ok = true;
     for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
@@ -559,7 +651,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w.nb > 0) {
         int lo, hi;
         key_range(row, w.lk, p, lo, hi);
+        uint32_t pk[kBN / 2];  // P of the block, packed for the MMA
+        // Sum of the rounded P of the last block, from its packed words.
+        auto add_rounded = [&]() {
+          uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int i = 0; i < kBN / 2; ++i)
+            acc[i & 3] = add2(acc[i & 3], f2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
+          float b0, b1;
+          f2_split(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), b0, b1);
+          l_rnd += b0 + b1;
+        };
         for (int j = 0; j < w.nb; ++j) {
+          if (kRsum == 3 && j > 0) add_rounded();
           ok = mbar_wait(&sm.s_full[t], scnt & 1, g);
           if (!ok) break;
           ++scnt;
@@ -594,66 +698,56 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_rnd *= alpha;
           const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
           const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
-          // P = 2^(s * scale * log2e - m); exact and rounded row sums in four
-          // independent packed accumulators each.
+          // P = 2^(s * scale * log2e - m); exact (and rounded) row sums in
+          // four independent packed accumulators each.
           uint64_t rs2[4] = {0, 0, 0, 0}, rr2[4] = {0, 0, 0, 0};
-          uint32_t pk[kBN / 2];
+          float rrs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          // Rescale the accumulator when the running max moved.  The previous
+          // P.V of this tile has completed: it was issued before this S.
+          auto rescale_o = [&]() {
+            const bool need = (j > 0) && (alpha != 1.f);
+            if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int q2 = 0; q2 < kBN / 2; ++q2) {
-            const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
-            float p0, p1;
-            if ((q2 & 7) >= 8 - kEmuPairsPer8) {
-              f2_split(exp2_poly2(x2), p0, p1);
-            } else {
-              float x0, x1;
-              f2_split(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t raw[32];
+                tmem_ld32(tO + c * 32, raw);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+                tmem_st32(tO + c * 32, raw);
+              }
             }
-            rs2[q2 & 3] = add2(rs2[q2 & 3], f2(p0, p1));
-            if (FP8) {
-              const uint16_t e = pack_e4m3x2(p0, p1);
-              if (q2 & 1) pk[q2 >> 1] |= (uint32_t)e << 16;
-              else pk[q2 >> 1] = e;
-              uint32_t h;
-              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(e));
-              float h0, h1;
-              asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-                  : "=f"(h0), "=f"(h1)
-                  : "r"(h));
-              rr2[q2 & 3] = add2(rr2[q2 & 3], f2(h0, h1));
-            } else {
-              const uint32_t b = pack_bf16x2(p0, p1);
-              pk[q2] = b;
-              rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
-            }
-          }
-          if (FP8) {
-            tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+          };
+          if (kSplitP) {
+#pragma unroll
+            for (int q2 = 0; q2 < kSplitKeys / 2; ++q2) p_pair<FP8, kRsumInline>(q2, sr, sc2, nm2, rs2, rr2, rrs, pk);
+            // bf16: one key pair per TMEM column; e4m3: two pairs
+            tmem_st_cols<0, (FP8 ? kSplitKeys / 4 : kSplitKeys / 2)>(tS, pk);
+            rescale_o();
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.p_half[t]);
+#pragma unroll
+            for (int q2 = kSplitKeys / 2; q2 < kBN / 2; ++q2) p_pair<FP8, kRsumInline>(q2, sr, sc2, nm2, rs2, rr2, rrs, pk);
+            tmem_st_cols<(FP8 ? kSplitKeys / 4 : kSplitKeys / 2), (FP8 ? kBN / 4 : kBN / 2)>(tS, pk);
           } else {
+#pragma unroll
+            for (int q2 = 0; q2 < kBN / 2; ++q2) p_pair<FP8, kRsumInline>(q2, sr, sc2, nm2, rs2, rr2, rrs, pk);
             tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-            tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            if (!FP8) tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            rescale_o();
           }
           {
             const uint64_t a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
-            const uint64_t b = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
-            float a0, a1, b0, b1;
+            float a0, a1;
             f2_split(a, a0, a1);
-            f2_split(b, b0, b1);
             l_run += a0 + a1;
-            l_rnd += b0 + b1;
-          }
-          // Rescale the accumulator when the running max moved.  The previous
-          // P.V of this tile has completed: it was issued before this S.
-          const bool need = (j > 0) && (alpha != 1.f);
-          if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t raw[32];
-              tmem_ld32(tO + c * 32, raw);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-              tmem_st32(tO + c * 32, raw);
+            if (kRsum == 1) {
+              const uint64_t b = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
+              float b0, b1;
+              f2_split(b, b0, b1);
+              l_rnd += b0 + b1;
+            } else if (kRsum == 2) {
+              l_rnd += ((rrs[0] + rrs[1]) + (rrs[2] + rrs[3])) + ((rrs[4] + rrs[5]) + (rrs[6] + rrs[7]));
             }
           }
           tmem_st_wait();
@@ -661,6 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&sm.p_full[t]);
         }
         if (!ok) break;
+        if (kRsum == 3) add_rounded();
         // Hand the row statistics of this unit to the epilogue warpgroup, once
         // it has taken the previous unit's: a unit of one K/V block can finish
         // while the epilogue is still on the other tile of the unit before.
@@ -670,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm.st_m[t][r] = m_run;
         sm.st_l[t][r] = l_run;
-        sm.st_r[t][r] = l_rnd;
+        sm.st_r[t][r] = kRsum != 0 ? l_rnd : l_run;
         mbar_arrive(&sm.st_full[t]);
         ++nunit;
       }

@@ -261,6 +261,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+// registers -> TMEM, 32 lanes x 8 columns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// registers r[C0..C1) -> TMEM columns [C0, C1) of taddr (C1 - C0 a multiple of 8).
+template <int C0, int C1>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* r) {
+  static_assert((C1 - C0) % 8 == 0, "column range must be a multiple of 8");
+  if constexpr (C1 - C0 >= 32) {
+    tmem_st32(taddr + C0, *reinterpret_cast<const uint32_t(*)[32]>(r + C0));
+    tmem_st_cols<C0 + 32, C1>(taddr, r);
+  } else if constexpr (C1 - C0 >= 16) {
+    tmem_st16(taddr + C0, r + C0);
+    tmem_st_cols<C0 + 16, C1>(taddr, r);
+  } else if constexpr (C1 - C0 >= 8) {
+    tmem_st8(taddr + C0, r + C0);
+  }
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
