@@ -6,12 +6,14 @@ One step = one pass of the whole path over one batch of synthetic inputs:
      P.V, epilogue);
   2. paged decode: MQA, B=64 sequences, Hq=32, Hkv=1, D=128, lengths uniform in
      [512, 8192], 16-token pages behind a permuted block table
-     (attn_decode_paged: split + combine).
+     (attn_decode_paged: split + combine), against three K/V pools of that
+     batch in turn (the caches of three layers, 142 MB each).
 
 The headline ``value`` is prefill TFLOP/s (FLOPs counted as the causal mask
-requires); decode HBM GB/s is reported beside it.  Both come from CUDA events
-recorded around each kernel launch on the launching stream inside the timed
-region.  ``--gpus N`` under torchrun runs N independent replicas (the path has
+requires); decode HBM GB/s is reported beside it, per call of the second and
+third pools, which run back to back, and (``isolated``) for the first pool's
+call alone after an L2 flush.  Both come from CUDA events recorded on the
+launching stream inside the timed region.  ``--gpus N`` under torchrun runs N independent replicas (the path has
 no exchange step), times on the device and takes the max over ranks.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
@@ -43,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sources they were taken on (sha256 prefix of the files); a changed kernel
 # reports null until it is captured again.
 PROFILED_TRAFFIC = {
-    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "5d4bea9f89ab10b5",
-                "bytes": 312_252_928 + 97_561_600, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
-    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "f9baebc778a8a9a4",
-               "bytes": 147_916_544 + 4_712_960, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
+    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "83de6c90a5a1b063",
+                "bytes": 338_999_552 + 97_430_272, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
+    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "c50c9c107548e741",
+               "bytes": 147_881_472 + 4_232_704, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
 }
 
 
@@ -59,6 +61,7 @@ def profiled_traffic(kernel: str):
             h.update(fh.read())
     return entry["bytes"] if h.hexdigest()[:16] == entry["sha"] else None
 L2_FLUSH_BYTES = 256 << 20
+DECODE_LAYERS = 3  # K/V pools decoded per step
 
 
 def parse_args(argv=None):
@@ -229,6 +232,15 @@ def run_ours(args):
     dlse = torch.empty(dq.shape[:2], dtype=torch.float32, device=dev)
     ws = torch.empty(attn.attn_decode_workspace_bytes(DECODE.B, DECODE.Hq, kv.max_pages, DECODE.D),
                      dtype=torch.uint8, device=dev)
+    # Two more K/V pools of the same batch (same lengths and block table, their
+    # own values), as the caches of further layers: each step decodes the
+    # batch against all DECODE_LAYERS pools in turn.
+    g_pool = torch.Generator(device=dev)
+    g_pool.manual_seed(seed_of(2) + 1)
+    pools = [(dkp, dvp)] + [
+        (torch.randn(dkp.shape, generator=g_pool, device=dev).to(torch.bfloat16),
+         torch.randn(dvp.shape, generator=g_pool, device=dev).to(torch.bfloat16))
+        for _ in range(DECODE_LAYERS - 1)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_rd = torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -244,11 +256,17 @@ def run_ours(args):
         # to HBM here rather than during the decode.
         flush.zero_()
         flush_rd.view(torch.int32).sum(dtype=torch.int32)
+        # Layer 0 alone after the flush (isolated call), then the other layers
+        # back to back: their pools were last read a step ago, with the
+        # prefill, the flush and the other pools (> L2 each) read since.
         if ev is not None:
             ev[2].record(stream)
-        attn.attn_decode_paged(dq, dkp, dvp, dbt, dsl, DECODE.scale, o=do, lse=dlse, workspace=ws)
+        for li, (kp, vp) in enumerate(pools):
+            attn.attn_decode_paged(dq, kp, vp, dbt, dsl, DECODE.scale, o=do, lse=dlse, workspace=ws)
+            if ev is not None and li == 0:
+                ev[3].record(stream)
         if ev is not None:
-            ev[3].record(stream)
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -257,7 +275,7 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"kernel status {attn.attn_status_str(st)} during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
@@ -280,7 +298,9 @@ def run_ours(args):
 
     region_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     pre_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world, dev)
-    dec_ms = max_over_ranks(sum(e[2].elapsed_time(e[3]) for e in evs), world, dev)
+    dec1_ms = max_over_ranks(sum(e[2].elapsed_time(e[3]) for e in evs), world, dev)
+    # back-to-back calls: layers 1.. of every step, per call
+    dec_ms = max_over_ranks(sum(e[3].elapsed_time(e[4]) for e in evs), world, dev) / (DECODE_LAYERS - 1)
     K = args.steps
     pf = prefill_flops(PREFILL)
     db = decode_bytes(DECODE, kv.seq_lens.tolist())
@@ -289,6 +309,7 @@ def run_ours(args):
     per_launch_pre_ms = pre_ms / K
     achieved_pre = pf / (per_launch_pre_ms / 1e3) / 1e12        # per GPU, per launch
     achieved_dec = db / (dec_ms / K / 1e3) / 1e9
+    achieved_dec1 = db / (dec1_ms / K / 1e3) / 1e9
 
     # ---- end to end through the public API with host buffers
     pin = lambda t: t.pin_memory()  # noqa: E731
@@ -360,7 +381,9 @@ def run_ours(args):
         "config": {
             "workload": "prefill gqa_causal B4 Hq32 Hkv8 L4096 D128 + paged decode mqa B64 Hq32 Hkv1 D128 len[512,8192] page16",
             "prefill": PREFILL.name, "decode": DECODE.name,
-            "l2": "prefill inputs 201 MB > L2; before each decode a 256 MB buffer is written, then another read",
+            "l2": ("prefill inputs 201 MB > L2; decode: a 256 MB buffer is written, then another read, before "
+                   f"the first of {DECODE_LAYERS} K/V pools (142 MB each, > L2) of the batch; the pools are decoded "
+                   "in turn, the later ones back to back (the decode figures), the first alone (isolated)"),
             "parallelism": f"replicas{world}",
         },
         "roofline": {
@@ -375,14 +398,18 @@ def run_ours(args):
         "decode": {
             "value": round(dec_gbs, 1), "unit": "GB/s", "workload": DECODE.name,
             "us_per_call": round(dec_ms / K * 1e3, 2),
+            "timing": f"calls on K/V pools 2..{DECODE_LAYERS} of each step, back to back, per call",
             "roofline": {"bound": "hbm", "achieved": round(achieved_dec, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(achieved_dec / peaks["hbm_gbs"], 4),
                          "peak_source": f"{peak_src} hbm_gbs", "traffic": profiled_traffic("decode"),
                          "algorithmic_bytes": db},
+            "isolated": {"us_per_call": round(dec1_ms / K * 1e3, 2), "GB/s": round(achieved_dec1, 1),
+                         "frac": round(achieved_dec1 / peaks["hbm_gbs"], 4),
+                         "timing": "the first pool's call alone, after the L2 flush, events around it"},
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * K,
+        "gpu_launches": (1 + 2 * DECODE_LAYERS) * K,  # prefill + (split, combine) per decode call
         "clocks": clk,
         "cpu_baseline": cpu,
         "workloads": extra,
