@@ -203,6 +203,10 @@ struct CombineParams {
 // segment s's log2-sum-exp while every lane reads its 4 features of up to 8
 // partials at once.
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
+  // The next decode's split kernel (a programmatic dependent) may launch and
+  // set up while this grid runs; it waits for this grid before reading or
+  // writing global memory.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);  // output row: (b, h, token)
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hq * p.q_len) {
@@ -297,14 +301,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t base = smem_u32(smem_raw);
+  // This grid is launched as a programmatic dependent of the kernel before it
+  // in the stream, so that its launch and the set-up below (barriers, TMEM)
+  // overlap that kernel's tail.  That kernel may write any of the inputs or
+  // read the workspace, so nothing global is touched before
+  // griddepcontrol.wait.
   if (base & 1023u) {  // the layout below needs a 1024-byte aligned base
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) atomicExch(p.status, kErrBounds);
     return;
   }
-  // The page counts of the first 64 sequences are requested before anything
-  // else; barrier set-up and the TMEM allocation run while they are in flight.
-  const int sl0 = lane < p.B ? p.seq_lens[lane] : 0;
-  const int sl1 = lane + 32 < p.B ? p.seq_lens[lane + 32] : 0;
   const uint32_t q_slot = 2u * p.q_half;
   const uint32_t nqs = (uint32_t)p.q_slots, nst = (uint32_t)p.stages;
   const uint32_t s_q = base;                       // query slots
@@ -332,6 +338,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int sl0 = lane < p.B ? p.seq_lens[lane] : 0;
+  const int sl1 = lane + 32 < p.B ? p.seq_lens[lane + 32] : 0;
   // Total pages T of the batch and this CTA's share.  Every warp sums the
   // page counts itself, lane l taking sequences l, l + 32, ... (independent
   // loads, then a shuffle reduction), so no warp waits for another.
@@ -793,8 +802,18 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (!encode_q(&tq, a.q, a.B * a.Hq * q_len, rows) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
         !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv))
       return fail_cuda("decode: tensor map", cudaErrorInvalidValue);
-    decode_split_kernel<<<split_grid, kThreads, smem, stream>>>(tq, tk, tv, sp);
-    err = cudaGetLastError();
+    cudaLaunchConfig_t scfg{};
+    scfg.gridDim = dim3(split_grid);
+    scfg.blockDim = dim3(kThreads);
+    scfg.dynamicSmemBytes = smem;
+    scfg.stream = stream;
+    cudaLaunchAttribute sattr[1];
+    sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    sattr[0].val.programmaticStreamSerializationAllowed = 1;
+    scfg.attrs = sattr;
+    scfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&scfg, decode_split_kernel, tq, tk, tv, sp);
+    if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return fail_cuda("decode: split launch", err);
   }
   CombineParams cp{};
