@@ -503,23 +503,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (!ok) break;
         ++n_q;
         const uint32_t q_addr = s_q + qs * q_slot;
+        // S of block jj of the segment; the segment's last S is the last
+        // reader of its query slot, which is then released.
+        auto s_block = [&](int jj) {
+          const uint32_t x = n_blk + jj;
+          tc_fence_after();
+          issue_s(x, q_addr, min(kBlkPages, pg_hi - (pg_lo + jj * kBlkPages)));
+          tc_commit(&sm.s_full[x & 1]);
+          if (jj == nb - 1) tc_commit(&sm.q_empty[qs]);
+        };
         for (int j = 0; j < nb && ok; ++j) {
           const uint32_t gb = n_blk + j;
           if (j == 0) {
             ok = mbar_wait(&sm.kv_full[gb % nst], (gb / nst) & 1, g);
             if (!ok) break;
-            tc_fence_after();
-            issue_s(gb, q_addr, min(kBlkPages, pg_hi - pg_lo));
-            tc_commit(&sm.s_full[gb & 1]);
+            s_block(0);
           }
-          if (j + 1 < nb) {  // next block's scores while this block's softmax runs
-            const uint32_t gn = gb + 1;
-            ok = mbar_wait(&sm.kv_full[gn % nst], (gn / nst) & 1, g);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(gn, q_addr, min(kBlkPages, pg_hi - (pg_lo + (j + 1) * kBlkPages)));
-            tc_commit(&sm.s_full[gn & 1]);
-          }
+          // The next block's scores go first, so that they are ready when this
+          // block's softmax ends, but only if its K/V has already landed:
+          // waiting for it here would hold back this block's P V and with it
+          // the release of its stage, leaving the producer one load in flight.
+          const bool has_next = j + 1 < nb;
+          const uint32_t gn = gb + 1;
+          const bool s_first = has_next && mbar_test(&sm.kv_full[gn % nst], (gn / nst) & 1);
+          if (s_first) s_block(j + 1);
           ok = mbar_wait(&sm.p_full[gb & 1], (gb >> 1) & 1, g);
           if (!ok) break;
           if (j == 0 && n_seg > 0) {
@@ -530,10 +537,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0);
           tc_commit(&sm.kv_empty[gb % nst]);
           tc_commit(&sm.pv_done);
+          if (has_next && !s_first) {
+            ok = mbar_wait(&sm.kv_full[gn % nst], (gn / nst) & 1, g);
+            if (!ok) break;
+            s_block(j + 1);
+          }
         }
         if (!ok) break;
         tc_commit(&sm.o_full);
-        tc_commit(&sm.q_empty[qs]);
         n_blk += nb;
         ++n_seg;
       }
