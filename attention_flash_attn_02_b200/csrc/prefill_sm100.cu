@@ -66,7 +66,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 #define ATTN_EMU_PAIRS_PER8 0
 #endif
 #ifndef ATTN_EMU_PAIRS_PER8_FP8
-#define ATTN_EMU_PAIRS_PER8_FP8 2
+#define ATTN_EMU_PAIRS_PER8_FP8 0
 #endif
 template <bool FP8>
 constexpr int kEmuPairsPer8 = FP8 ? ATTN_EMU_PAIRS_PER8_FP8 : ATTN_EMU_PAIRS_PER8;
