@@ -57,13 +57,25 @@ def up_to_date() -> bool:
 PREFILL_LAUNCH_REGS = 128
 
 
+# Kernels whose inner loops must not touch local memory: a spill there costs
+# more than any tuning gains, so the build refuses it.
+NO_SPILL_KERNELS = ("prefill_kernel", "decode_split_kernel", "bwd_kernel")
+
+
 def check_register_counts(ptxas_log: str) -> None:
+    """Checks ptxas -v output: the prefill kernels launch with
+    PREFILL_LAUNCH_REGS registers and the hot kernels do not spill."""
     entry = None
     seen = 0
     for line in ptxas_log.splitlines():
         m = re.search(r"Compiling entry function '([^']+)'", line)
         if m:
             entry = m.group(1)
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m and entry and any(k in entry for k in NO_SPILL_KERNELS):
+            if int(m.group(1)) or int(m.group(2)):
+                raise RuntimeError(f"{entry}: spills ({line.strip()})")
             continue
         m = re.search(r"Used (\d+) registers", line)
         if m and entry and "prefill_kernel" in entry:

@@ -168,3 +168,27 @@ def test_missing_library_fails_loudly(tmp_path):
             attn.load(str(tmp_path / "nope.so"))
     finally:
         attn._lib = saved
+
+
+def _ptxas_log(kernel, regs=128, spill_st=0, spill_ld=0):
+    return (f"ptxas info    : Compiling entry function '_ZN4attn{kernel}Ev' for 'sm_100a'\n"
+            f"ptxas info    : Function properties for _ZN4attn{kernel}Ev\n"
+            f"    0 bytes stack frame, {spill_st} bytes spill stores, {spill_ld} bytes spill loads\n"
+            f"ptxas info    : Used {regs} registers, used 2 barriers\n")
+
+
+def test_build_check_accepts_clean_prefill_log():
+    from attention_flash_attn_02_b200.build import check_register_counts
+    check_register_counts(_ptxas_log("14prefill_kernel") + _ptxas_log("19decode_split_kernel", regs=148))
+
+
+def test_build_check_rejects_wrong_launch_count_and_spills():
+    from attention_flash_attn_02_b200.build import check_register_counts
+    with pytest.raises(RuntimeError, match="registers"):
+        check_register_counts(_ptxas_log("14prefill_kernel", regs=168))
+    with pytest.raises(RuntimeError, match="spills"):
+        check_register_counts(_ptxas_log("14prefill_kernel", spill_st=44, spill_ld=40))
+    with pytest.raises(RuntimeError, match="spills"):
+        check_register_counts(_ptxas_log("14prefill_kernel") + _ptxas_log("10bwd_kernel", spill_st=8))
+    with pytest.raises(RuntimeError, match="no prefill"):
+        check_register_counts(_ptxas_log("19decode_split_kernel"))
