@@ -77,22 +77,16 @@ constexpr int kEmuPairsPer8 = FP8 ? ATTN_EMU_PAIRS_PER8_FP8 : ATTN_EMU_PAIRS_PER
 #define ATTN_SPLIT_P 6
 #endif
 constexpr bool kSplitP = ATTN_SPLIT_P != 0;
-#ifndef ATTN_EARLY_Q
-#define ATTN_EARLY_Q 1
-#endif
-constexpr bool kEarlyQ = ATTN_EARLY_Q != 0;
 constexpr int kSplitKeys = ATTN_SPLIT_P * 16;
 static_assert(ATTN_SPLIT_P == 0 || (ATTN_SPLIT_P % 2 == 0 && ATTN_SPLIT_P < 8), "split at 32, 64 or 96 keys");
 // bf16 path: O is normalised by the sum of the bf16-rounded P that the MMA
-// multiplies (1: halves unpacked by shift and mask, added in pairs; 2: each
-// half added by a mixed-precision bf16 + f32 add) or by the exact fp32 row
-// sum (0); 3: as 1, but summed from the packed words after P has been handed
-// to the MMA warp, while the warp waits for its next S.  On rows of a few keys the two sums differ by up to 2^-10, which
-// with the bf16 rounding of O can exceed 1e-2 absolute.  The e4m3 path always
-// uses the rounded sum.
+// multiplies (1) or by the exact fp32 row sum (0).  On rows of a few keys the
+// two sums differ by up to 2^-10, which with the bf16 rounding of O can exceed
+// 1e-2 absolute.  The e4m3 path always uses the rounded sum.
 #ifndef ATTN_ROUNDED_SUM
 #define ATTN_ROUNDED_SUM 1
 #endif
+static_assert(ATTN_ROUNDED_SUM == 0 || ATTN_ROUNDED_SUM == 1, "row-sum mode 0 or 1");
 
 template <int D, bool FP8>
 struct Cfg {
@@ -260,10 +254,9 @@ static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserv
 // ex2, or for kEmuPairsPer8 of every 8 pairs the FMA-pipe polynomial), packed
 // for the MMA, added to the exact row sum and, with RSUM, to the sum of the
 // rounded values.  e4m3 pairs go two to a 32-bit word.
-template <bool FP8, int RSUM>
+template <bool FP8, bool RSUM>
 __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
-                                       uint64_t (&rs2)[4], uint64_t (&rr2)[4], float (&rrs)[8],
-                                       uint32_t (&pk)[kBN / 2]) {
+                                       uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2]) {
   const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
   float p0, p1;
   if ((q2 & 7) >= 8 - kEmuPairsPer8<FP8>) {
@@ -289,14 +282,7 @@ __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64
   } else {
     const uint32_t b = pack_bf16x2(p0, p1);
     pk[q2] = b;
-    if (RSUM == 1) {
-      rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
-    } else if (RSUM == 2) {
-      asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-          "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
-          : "+f"(rrs[2 * (q2 & 3)]), "+f"(rrs[2 * (q2 & 3) + 1])
-          : "r"(b));
-    }
+    if (RSUM) rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
   }
 }
 
@@ -548,10 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // while this unit's last softmax and P V run.
         issue_s(0, kv_addr0 + sk * C::TILE_BYTES);
         tc_commit(&sm.s_full[0]);
-        if (kEarlyQ && w.nb == 1) tc_commit(&sm.q_empty[0]);
+        if (w.nb == 1) tc_commit(&sm.q_empty[0]);
         issue_s(1, kv_addr0 + sk * C::TILE_BYTES);
         tc_commit(&sm.s_full[1]);
-        if (kEarlyQ && w.nb == 1) tc_commit(&sm.q_empty[1]);
+        if (w.nb == 1) tc_commit(&sm.q_empty[1]);
         tc_commit(&sm.kv_empty[sk]);
         for (int j = 0; j < w.nb && ok; ++j) {
           const uint32_t sv = seq % C::NS;
@@ -605,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               issue_s(t, kv_addr0 + skn * C::TILE_BYTES);
               tc_commit(&sm.s_full[t]);
-              if (kEarlyQ && j + 2 == w.nb) tc_commit(&sm.q_empty[t]);
+              if (j + 2 == w.nb) tc_commit(&sm.q_empty[t]);
             }
           }
           if (!ok) break;
@@ -617,10 +603,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        if (!kEarlyQ) {
-          tc_commit(&sm.q_empty[0]);
-          tc_commit(&sm.q_empty[1]);
-        }
         ++nunit;
       }
       // Drain: all issued MMAs complete before TMEM is released.
@@ -638,8 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + (t == 0 ? C::TM_S0 : C::TM_S1) + lane_off;
     const uint32_t tO = tmem + (t == 0 ? C::TM_O0 : C::TM_O1) + lane_off;
     const float sl2 = p.scale_log2;
-    constexpr int kRsum = FP8 ? 1 : ATTN_ROUNDED_SUM;
-    constexpr int kRsumInline = kRsum == 3 ? 0 : kRsum;
+    constexpr bool kRsum = FP8 || ATTN_ROUNDED_SUM;
     uint32_t scnt = 0, nunit = 0;
     bool ok = true;
     for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
@@ -651,19 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w.nb > 0) {
         int lo, hi;
         key_range(row, w.lk, p, lo, hi);
-        uint32_t pk[kBN / 2];  // P of the block, packed for the MMA
-        // Sum of the rounded P of the last block, from its packed words.
-        auto add_rounded = [&]() {
-          uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int i = 0; i < kBN / 2; ++i)
-            acc[i & 3] = add2(acc[i & 3], f2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
-          float b0, b1;
-          f2_split(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), b0, b1);
-          l_rnd += b0 + b1;
-        };
         for (int j = 0; j < w.nb; ++j) {
-          if (kRsum == 3 && j > 0) add_rounded();
           ok = mbar_wait(&sm.s_full[t], scnt & 1, g);
           if (!ok) break;
           ++scnt;
@@ -701,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // P = 2^(s * scale * log2e - m); exact (and rounded) row sums in
           // four independent packed accumulators each.
           uint64_t rs2[4] = {0, 0, 0, 0}, rr2[4] = {0, 0, 0, 0};
-          float rrs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          uint32_t pk[kBN / 2];  // P of the block, packed for the MMA
           // Rescale the accumulator when the running max moved.  The previous
           // P.V of this tile has completed: it was issued before this S.
           auto rescale_o = [&]() {
@@ -719,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           };
           if (kSplitP) {
 #pragma unroll
-            for (int q2 = 0; q2 < kSplitKeys / 2; ++q2) p_pair<FP8, kRsumInline>(q2, sr, sc2, nm2, rs2, rr2, rrs, pk);
+            for (int q2 = 0; q2 < kSplitKeys / 2; ++q2) p_pair<FP8, kRsum>(q2, sr, sc2, nm2, rs2, rr2, pk);
             // bf16: one key pair per TMEM column; e4m3: two pairs
             tmem_st_cols<0, (FP8 ? kSplitKeys / 4 : kSplitKeys / 2)>(tS, pk);
             rescale_o();
@@ -727,11 +696,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&sm.p_half[t]);
 #pragma unroll
-            for (int q2 = kSplitKeys / 2; q2 < kBN / 2; ++q2) p_pair<FP8, kRsumInline>(q2, sr, sc2, nm2, rs2, rr2, rrs, pk);
+            for (int q2 = kSplitKeys / 2; q2 < kBN / 2; ++q2) p_pair<FP8, kRsum>(q2, sr, sc2, nm2, rs2, rr2, pk);
             tmem_st_cols<(FP8 ? kSplitKeys / 4 : kSplitKeys / 2), (FP8 ? kBN / 4 : kBN / 2)>(tS, pk);
           } else {
 #pragma unroll
-            for (int q2 = 0; q2 < kBN / 2; ++q2) p_pair<FP8, kRsumInline>(q2, sr, sc2, nm2, rs2, rr2, rrs, pk);
+            for (int q2 = 0; q2 < kBN / 2; ++q2) p_pair<FP8, kRsum>(q2, sr, sc2, nm2, rs2, rr2, pk);
             tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
             if (!FP8) tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
             rescale_o();
@@ -741,13 +710,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             float a0, a1;
             f2_split(a, a0, a1);
             l_run += a0 + a1;
-            if (kRsum == 1) {
+            if (kRsum) {
               const uint64_t b = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
               float b0, b1;
               f2_split(b, b0, b1);
               l_rnd += b0 + b1;
-            } else if (kRsum == 2) {
-              l_rnd += ((rrs[0] + rrs[1]) + (rrs[2] + rrs[3])) + ((rrs[4] + rrs[5]) + (rrs[6] + rrs[7]));
             }
           }
           tmem_st_wait();
@@ -755,7 +722,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&sm.p_full[t]);
         }
         if (!ok) break;
-        if (kRsum == 3) add_rounded();
         // Hand the row statistics of this unit to the epilogue warpgroup, once
         // it has taken the previous unit's: a unit of one K/V block can finish
         // while the epilogue is still on the other tile of the unit before.
@@ -765,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm.st_m[t][r] = m_run;
         sm.st_l[t][r] = l_run;
-        sm.st_r[t][r] = kRsum != 0 ? l_rnd : l_run;
+        sm.st_r[t][r] = kRsum ? l_rnd : l_run;
         mbar_arrive(&sm.st_full[t]);
         ++nunit;
       }
