@@ -120,10 +120,13 @@ def measured_peaks():
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons of the GPU under test with
-    nvidia-smi every 200 ms from a background thread while the timed region
-    runs.  The device is matched by UUID, else by index, else it is the only
-    GPU nvidia-smi lists."""
+    """Samples the SM clock and the throttle reasons of the GPU under test
+    from a background thread while the timed region runs: through NVML every
+    5 ms, so that a region of a few tens of milliseconds still gets samples,
+    else with nvidia-smi every 200 ms.  Only samples taken between
+    ``begin()`` and ``end()`` (host time around the region, whose GPU work
+    the final synchronize bounds) are reported.  The device is matched by
+    UUID, else by index, else it is the only GPU listed."""
 
     FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -132,51 +135,105 @@ class ClockSampler:
 
     def __init__(self, uuid: str, index: int):
         self.uuid = (uuid or "").lower().replace("gpu-", "").replace("-", "")
-        self.index = str(index)
-        self.rows = []
+        self.index = index
+        self.rows = []          # (host time, sm MHz, max sm MHz, set of reasons)
+        self.source = None
         self._stop = None
         self._thread = None
+        self._first = None
+        self.t0 = self.t1 = None
 
-    def _poll(self):
-        import threading  # noqa: F401
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        n = pynvml.nvmlDeviceGetCount()
+        handles = [pynvml.nvmlDeviceGetHandleByIndex(i) for i in range(n)]
+        norm = lambda u: (u.decode() if isinstance(u, bytes) else u).lower().replace("gpu-", "").replace("-", "")  # noqa: E731
+        for h in handles:
+            if self.uuid and norm(pynvml.nvmlDeviceGetUUID(h)) == self.uuid:
+                return pynvml, h
+        if n == 1:
+            return pynvml, handles[0]
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll_nvml(self, pynvml, h):
+        get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = [getattr(pynvml, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                getattr(pynvml, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                getattr(pynvml, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                getattr(pynvml, "nvmlClocksEventReasonSwPowerCap", 0x4)]
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            t = time.perf_counter()
+            sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            r = get_reasons(h)
+            self.rows.append((t, float(sm), float(mx), {self.REASONS[i] for i in range(4) if r & bits[i]}))
+            self._first.set()
+            self._stop.wait(0.005)
+
+    def _poll_smi(self):
         while not self._stop.is_set():
             try:
+                t = time.perf_counter()
                 out = subprocess.run(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits"],
                                      capture_output=True, text=True, timeout=5).stdout
-                for line in out.splitlines():
-                    parts = [x.strip() for x in line.split(",")]
-                    if len(parts) >= 10:
-                        self.rows.append(parts)
+                rows = [[x.strip() for x in line.split(",")] for line in out.splitlines()]
+                rows = [r for r in rows if len(r) >= 10]
+                norm = lambda u: u.lower().replace("gpu-", "").replace("-", "")  # noqa: E731
+                mine = [r for r in rows if self.uuid and norm(r[1]) == self.uuid]
+                if not mine:
+                    mine = rows if len(rows) == 1 else [r for r in rows if r[0] == str(self.index)]
+                num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None  # noqa: E731
+                for r in mine:
+                    if num(r[2]) is not None:
+                        self.rows.append((t, num(r[2]), num(r[3]),
+                                          {self.REASONS[i] for i in range(4) if r[6 + i].lower() == "active"}))
             except Exception:
                 pass
+            self._first.set()
             self._stop.wait(0.2)
+
+    def _run(self):
+        try:
+            pynvml, h = self._nvml_handle()
+            self.source = "nvml, 5 ms"
+            self._poll_nvml(pynvml, h)
+        except Exception:
+            self.source = "nvidia-smi, 200 ms"
+            self._poll_smi()
 
     def start(self):
         import threading
         self._stop = threading.Event()
-        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._first = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
+        self._first.wait(timeout=5)  # the first sample precedes the region
+
+    def begin(self):
+        self.t0 = time.perf_counter()
+
+    def end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
         if self._thread is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not sampled"], "samples": 0}
         self._stop.set()
         self._thread.join(timeout=10)
-        rows = self.rows
-        norm = lambda u: u.lower().replace("gpu-", "").replace("-", "")  # noqa: E731
-        mine = [r for r in rows if self.uuid and norm(r[1]) == self.uuid]
+        t0 = self.t0 if self.t0 is not None else float("-inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        mine = [r for r in self.rows if t0 <= r[0] <= t1]
         if not mine:
-            indices = {r[0] for r in rows}
-            mine = rows if len(indices) == 1 else [r for r in rows if r[0] == self.index]
-        if not mine:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None  # noqa: E731
-        sm = [num(r[2]) for r in mine if num(r[2]) is not None]
-        mx = [num(r[3]) for r in mine if num(r[3]) is not None]
-        reasons = sorted({self.REASONS[i] for r in mine for i in range(4) if r[6 + i].lower() == "active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples in the timed region"],
+                    "samples": 0, "source": self.source}
+        sm = [r[1] for r in mine]
         load = [x for x in sm if x > 500] or sm
-        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(mine)}
+        return {"sm_mhz": statistics.median(load), "sm_min_mhz": min(load),
+                "sm_max_mhz": max(r[2] for r in mine if r[2] is not None),
+                "reasons": sorted(set().union(*(r[3] for r in mine))), "samples": len(mine),
+                "source": self.source}
 
 
 # ----------------------------------------------------------- CPU baseline
@@ -285,11 +342,13 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
+    clocks.begin()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
+    clocks.end()
     barrier(world)
     clk = clocks.stop()
     st = attn.attn_last_device_error()
