@@ -109,6 +109,23 @@ static_assert(two_fit(dec_smem_bytes(kMaxGroup * 128, 1, 2)), "the largest tile 
 // memory that a third CTA would fit on an SM (its allocation would wait).
 constexpr int kMinSmem = 233472 / (kCtasPerSm + 1) - 1024 + 16;
 
+// K/V pages are read once per call, so their TMA loads carry an L2
+// evict-first policy: they then do not push out the small data that is read
+// again (sequence lengths, the block table, the partials the combine reads).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_load_3d_evict_first(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                                        int c0, int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ int len_of(const int* seq_lens, int max_pages, int b) {
   const int n = seq_lens[b], cap = max_pages * kPage;
   return n < 0 ? 0 : (n > cap ? cap : n);
@@ -399,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     uint32_t n_blk = 0, n_q = 0;
     bool ok = !p.stall;
+    const uint64_t pol = l2_evict_first_policy();
     Segments seg(p, lo, hi, lane);
     while (seg.more() && ok) {
       int b, kvh, pg_lo, pg_hi, P;
@@ -441,10 +459,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               for (int i = 0; i < nv; ++i) {
                 const int tok = pid[i] * kPage;
                 const uint32_t d = dst + i * kPageHalf;
-                tma_load_3d(d, &tm_k, &sm.kv_full[st], 0, kvh, tok);
-                tma_load_3d(d + kHalf, &tm_k, &sm.kv_full[st], 64, kvh, tok);
-                tma_load_3d(d + 2 * kHalf, &tm_v, &sm.kv_full[st], 0, kvh, tok);
-                tma_load_3d(d + 3 * kHalf, &tm_v, &sm.kv_full[st], 64, kvh, tok);
+                tma_load_3d_evict_first(d, &tm_k, &sm.kv_full[st], 0, kvh, tok, pol);
+                tma_load_3d_evict_first(d + kHalf, &tm_k, &sm.kv_full[st], 64, kvh, tok, pol);
+                tma_load_3d_evict_first(d + 2 * kHalf, &tm_v, &sm.kv_full[st], 0, kvh, tok, pol);
+                tma_load_3d_evict_first(d + 3 * kHalf, &tm_v, &sm.kv_full[st], 64, kvh, tok, pol);
               }
             }
           }

@@ -47,8 +47,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PROFILED_TRAFFIC = {
     "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "9e739ca46748c6ba",
                 "bytes": 361_058_560 + 97_935_616, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
-    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "068650fbc2bea8d7",
-               "bytes": 147_897_600 + 3_990_528, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
+    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "bc446ec70993fe26",
+               "bytes": 147_640_832 + 4_014_848, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
 }
 
 
