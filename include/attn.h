@@ -2,7 +2,7 @@
  * attn.h -- C ABI of the B200 (sm_100a) fused attention library
  * (libattn_sm100.so).
  *
- * Two operations, both forward only, both on one GPU:
+ * Operations, all on one GPU:
  *
  *   attn_fwd / attn_fwd_fp8   fused, tiled scaled-dot-product attention
  *                             O = softmax(scale * Q K^T + mask) V, with the
@@ -13,7 +13,14 @@
  *   attn_decode_paged         one query token per sequence against a KV cache
  *                             held in fixed-size pages addressed through a
  *                             block table, split over the cache and merged by
- *                             log-sum-exp.
+ *                             log-sum-exp (attn_decode_paged_multi: the last
+ *                             q_len cached tokens; attn_decode_paged_noalloc:
+ *                             scratch inside the library).
+ *   attn_prefill_paged        a chunk of new tokens against the paged cache
+ *                             (chunked prefill), with attn_kv_append writing
+ *                             the chunk's K/V into its pages.
+ *   attn_bwd                  gradients dQ, dK, dV of attn_fwd, recomputing
+ *                             the weights from the forward's LSE.
  *
  * Sources (page title, section):
  *   - "003-注意力机制详解：从基础Attention到DeepSeek的优化策略" (lakecityint.com),
@@ -36,6 +43,10 @@
  *     status word per GPU, created when the library is loaded.
  *   - All launches are asynchronous on the caller's CUDA stream `stream`
  *     (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *     The decode kernels are launched as programmatic dependents of the
+ *     kernel before them in the stream: they may become resident and set up
+ *     early, but read and write no global memory until that kernel has
+ *     completed, so stream order holds as for a plain launch.
  *   - A call returns ATTN_OK once its kernels are enqueued.  Argument errors
  *     are detected on the host before anything is launched and return
  *     ATTN_ERR_INVALID / ATTN_ERR_UNSUPPORTED with nothing written.  A CUDA
