@@ -47,6 +47,11 @@ int fail_cuda(const char* where, cudaError_t err) {
   return ATTN_ERR_CUDA;
 }
 
+int fail_invalid(const char* msg) {
+  snprintf(g_msg, sizeof(g_msg), "%s", msg);
+  return ATTN_ERR_INVALID;
+}
+
 int debug_flags() { return g_debug_flags.load(); }
 unsigned long long wait_timeout_ns() { return g_timeout_ns.load(); }
 
@@ -114,11 +119,12 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq
   return decode_workspace_bytes(B, Hq, max_pages_per_seq, D);
 }
 
-namespace {
-int decode_checked(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
-                   const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int q_len, int D,
-                   int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
-                   size_t workspace_bytes, attn_stream_t stream) {
+namespace attn {
+// Every check of the decode arguments except the workspace: ATTN_OK to go on
+// (B == 0 included: nothing to launch), else the status to return.
+int validate_decode(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                    const int* seq_lens, const void* o, const float* lse, int B, int Hq, int Hkv, int q_len, int D,
+                    int page_size, int num_pages, int max_pages_per_seq, float scale) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages_per_seq < 0 ||
       q_len <= 0)
     return ATTN_ERR_INVALID;
@@ -132,6 +138,18 @@ int decode_checked(const void* q, const void* k_pages, const void* v_pages, cons
   if (num_pages > 0 && (!k_pages || !v_pages || !aligned16(k_pages) || !aligned16(v_pages)))
     return ATTN_ERR_INVALID;
   if (D != 128 || page_size != 16 || (Hq / Hkv) * q_len > 128) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+}  // namespace attn
+
+namespace {
+int decode_checked(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                   const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int q_len, int D,
+                   int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                   size_t workspace_bytes, attn_stream_t stream) {
+  const int st = validate_decode(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D,
+                                 page_size, num_pages, max_pages_per_seq, scale);
+  if (st != ATTN_OK || B == 0) return st;
   const int mp = max_pages_per_seq > 0 ? max_pages_per_seq : 1;
   const size_t need = attn_decode_workspace_bytes(B, Hq * q_len, mp, D);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_INVALID;

@@ -11,12 +11,24 @@
 // the library image, so the call itself allocates nothing.
 //
 // Costs of that choice, stated plainly:
-//   * every GPU that loads the library holds the array (kScratchBytes) until
-//     the process exits, whether or not the entry point is used;
+//   * the array (kScratchBytes) is device memory of the library's image.  The
+//     CUDA runtime loads this file's code and data onto a GPU when it is
+//     first needed there -- with lazy module loading (the default), at the
+//     first call of this entry point on that device, whose address look-up
+//     needs the array.  That first call per device therefore allocates the
+//     array and may synchronise: make it once at start-up, with the device
+//     current, outside any context that forbids allocation or
+//     synchronisation and before any stream capture (a call with B == 0 does
+//     only this set-up).  Every later call on that device allocates nothing,
+//     and the array stays until the process exits;
 //   * all calls share the one array and it keeps the last call's contents;
 //     two calls that overlap on the GPU (different streams without ordering
 //     between them) race on it and give wrong results;
-//   * sizes whose scratch would exceed the array are rejected.
+//   * sizes whose scratch would exceed the array are rejected;
+//   * the array's address is cached per device for the life of the process:
+//     after cudaDeviceReset the cached address is stale, and this entry point
+//     (like the rest of the library, which caches per-device state the same
+//     way) must not be called again in that process.
 // Nothing in the array has to start at zero: each call writes every partial
 // it later reads before reading it.
 #include <cstdio>
@@ -67,20 +79,23 @@ ATTN_API int attn_decode_paged_noalloc(const void* q, const void* k_pages, const
                                        const int* block_table, const int* seq_lens, void* o, float* lse, int B,
                                        int Hq, int Hkv, int D, int page_size, int num_pages, int max_pages_per_seq,
                                        float scale, attn_stream_t stream) {
-  if (B < 0 || Hq <= 0 || D <= 0 || max_pages_per_seq < 0) return ATTN_ERR_INVALID;
-  if (B == 0) return ATTN_OK;
+  // The same argument checks as attn_decode_paged, in the same order, so the
+  // two return the same status for the same arguments.
+  int st = validate_decode(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, 1, D, page_size,
+                           num_pages, max_pages_per_seq, scale);
+  if (st != ATTN_OK) return st;
+  // Set-up (first call per device, B == 0 included): the array's address.
+  void* scratch = nullptr;
+  st = scratch_for_current_device(&scratch);
+  if (st != ATTN_OK || B == 0) return st;
   const size_t need = attn_decode_workspace_bytes(B, Hq, max_pages_per_seq > 0 ? max_pages_per_seq : 1, D);
   if (need > kScratchBytes) {
-    // Too large for the fixed array: refuse before touching the GPU.
+    // Too large for the fixed array: refuse before launching anything.
     snprintf(g_noalloc_msg, sizeof(g_noalloc_msg),
              "attn_decode_paged_noalloc: these sizes need %zu bytes of scratch, the built-in array holds %zu",
              need, kScratchBytes);
-    fail_cuda(g_noalloc_msg, cudaErrorInvalidValue);
-    return ATTN_ERR_INVALID;
+    return fail_invalid(g_noalloc_msg);
   }
-  void* scratch = nullptr;
-  const int st = scratch_for_current_device(&scratch);
-  if (st != ATTN_OK) return st;
   return attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
                            num_pages, max_pages_per_seq, scale, scratch, kScratchBytes, stream);
 }

@@ -52,6 +52,12 @@ int sm_count();
 
 // Records a host-side failure for attn_last_error_message(); returns -3.
 int fail_cuda(const char* where, cudaError_t err);
+// Records an argument refusal for attn_last_error_message(); returns -1.
+int fail_invalid(const char* msg);
+// Checks of the decode arguments, workspace excepted (attn_api.cu).
+int validate_decode(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                    const int* seq_lens, const void* o, const float* lse, int B, int Hq, int Hkv, int q_len, int D,
+                    int page_size, int num_pages, int max_pages_per_seq, float scale);
 
 // Launchers: return a status code of include/attn.h.
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);

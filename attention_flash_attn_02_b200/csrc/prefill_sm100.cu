@@ -10,12 +10,13 @@
 // blocks wholly above the causal diagonal or before the sliding window are
 // never loaded (kler.cn page §一.2; window of the zeeklog page).
 //
-// B200 mapping (one persistent CTA per SM, 384 threads):
+// B200 mapping (one persistent CTA per SM, 512 threads in 4 warpgroups):
 //   warps 0-3   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 4-7   softmax warpgroup for Q tile 1
 //   warp  8     TMA producer: Q tiles, then K_j, V_j into a ring of stages
 //   warp  9     MMA issuer (one thread) + TMEM owner
-//   warps 10-11 idle (complete the third warpgroup)
+//   warps 10-11 idle (they complete the third warpgroup)
+//   warps 12-15 epilogue: O = acc / sum to bf16 and the LSE, per unit
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,..).
 // P (bf16 or e4m3) is written back over the first columns of its S buffer
 // and consumed from TMEM as the A operand of O += P V.
@@ -59,6 +60,21 @@ constexpr int kEpilogueRegs = 40;
 static_assert(2 * kSoftmaxRegs + kIssueRegs + kEpilogueRegs == 4 * kLaunchRegs,
               "register split must match the launch total");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// e4m3 tiles whose rows see few keys ("fine" tiles).  Rounding P to e4m3 (3
+// mantissa bits) moves each weight by up to 2^-4 relative; on a row of a
+// handful of keys that error does not average out and can reach ~6e-2 in O.
+// For a tile whose first row (the row that sees the fewest keys) sees fewer
+// than kFineKeys keys, the kernel therefore multiplies V by P in two parts:
+// h = e4m3(P) and the rounding residual e4m3(P - h), accumulated into the same
+// O, so each weight carries ~7 significant bits.  In those tiles P is scaled
+// by 2^kFineShift (the running max is kept exact, so P <= 2^8 <= 448, the
+// e4m3 maximum) so that residuals stay above e4m3's subnormal range; the
+// scale cancels in O / sum and is taken out of the LSE.  The residual lives in
+// TMEM columns [32, 64) of the tile's S buffer (P of 128 keys in e4m3 fills
+// columns [0, 32); all 128 columns of S are in registers by then).
+constexpr int kFineKeys = 512;
+constexpr float kFineShift = 8.0f;
+constexpr uint32_t kFineCol = 32;
 constexpr float kLn2 = 0.6931471805599453f;
 // Of every 8 pairs of exponentials, this many are computed by the FMA-pipe
 // polynomial instead of the MUFU ex2 unit (balances the two pipes).
@@ -139,6 +155,11 @@ struct Params {
 };
 
 constexpr int kPage = 16;  // tokens per page of a paged K/V pool
+
+template <int N>
+struct IntC {
+  static constexpr int value = N;
+};
 
 struct Unit {
   int bh[2];  // b * Hq + head of each tile
@@ -254,9 +275,12 @@ static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserv
 // ex2, or for kEmuPairsPer8 of every 8 pairs the FMA-pipe polynomial), packed
 // for the MMA, added to the exact row sum and, with RSUM, to the sum of the
 // rounded values.  e4m3 pairs go two to a 32-bit word.
-template <bool FP8, bool RSUM>
+// FINE (e4m3 only): also the residual e4m3(P - h) into pk_lo, and the sum of
+// h + residual, the weight the two products apply together.
+template <bool FP8, bool RSUM, bool FINE>
 __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
-                                       uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2]) {
+                                       uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
+                                       uint32_t (&pk_lo)[kBN / 4]) {
   const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
   float p0, p1;
   if ((q2 & 7) >= 8 - kEmuPairsPer8<FP8>) {
@@ -278,12 +302,60 @@ __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64
     asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
         : "=f"(h0), "=f"(h1)
         : "r"(h));
+    if (FINE) {
+      // P - h is exact in fp32 (h is P rounded to a 4-bit significand).
+      const uint16_t el = pack_e4m3x2(p0 - h0, p1 - h1);
+      if (q2 & 1) pk_lo[q2 >> 1] |= (uint32_t)el << 16;
+      else pk_lo[q2 >> 1] = el;
+      uint32_t hl;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hl) : "h"(el));
+      float l0, l1;
+      asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+          : "=f"(l0), "=f"(l1)
+          : "r"(hl));
+      h0 += l0;
+      h1 += l1;
+    }
     rr2[q2 & 3] = add2(rr2[q2 & 3], f2(h0, h1));
   } else {
     const uint32_t b = pack_bf16x2(p0, p1);
     pk[q2] = b;
     if (RSUM) rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
   }
+}
+
+template <bool FP8, bool RSUM, bool FINE, int Q_LO, int Q_HI>
+__device__ __forceinline__ void p_pairs(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2, uint64_t (&rs2)[4],
+                                        uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2], uint32_t (&pk_lo)[kBN / 4]) {
+#pragma unroll
+  for (int q2 = Q_LO; q2 < Q_HI; ++q2) p_pair<FP8, RSUM, FINE>(q2, sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+}
+
+// Fine e4m3 tiles: pairs [Q_LO, Q_HI) in chunks of 16 (32 keys), each chunk's
+// P and residual stored to TMEM at once (columns Q/2 on, at taddr and
+// taddr + kFineCol), so that the residual adds few live registers.
+template <bool RSUM, int Q_LO, int Q_HI>
+__device__ __forceinline__ void p_pairs_fine(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
+                                             uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
+                                             uint32_t (&pk_lo)[kBN / 4], uint32_t taddr) {
+  if constexpr (Q_LO < Q_HI) {
+    constexpr int QE = Q_LO + 16 < Q_HI ? Q_LO + 16 : Q_HI;
+    p_pairs<true, RSUM, true, Q_LO, QE>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+    tmem_st_cols<Q_LO / 2, QE / 2>(taddr, pk);
+    tmem_st_cols<Q_LO / 2, QE / 2>(taddr + kFineCol, pk_lo);
+    p_pairs_fine<RSUM, QE, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, taddr);
+  }
+}
+
+// Is tile t of unit w a "fine" e4m3 tile (its first row sees < kFineKeys keys)?
+template <bool FP8>
+__device__ __forceinline__ bool tile_fine(const Unit& w, int t, const Params& p) {
+  if (!FP8) return false;
+  const int m0 = w.m0_of(t);
+  if (m0 >= p.Lq) return false;
+  int lo, hi;
+  key_range(m0, w.lk, p, lo, hi);
+  return hi - lo < kFineKeys;
 }
 
 template <int D, bool FP8, bool PAGED>
@@ -506,11 +578,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_t (+)= P_t V: P from TMEM (over S_t), V MN-major, 128-byte column
       // groups BOX_BYTES apart, k-step kk = MMA_K keys of 128-byte rows.
       // k-steps [k_lo, k_hi) of the block's PV_KSTEPS.
-      auto issue_pv = [&](int t, uint32_t v_stage_addr, bool acc, int k_lo, int k_hi) {
+      // a_col: TMEM column of P within the S buffer (kFineCol: the residual
+      // of a fine e4m3 tile).
+      auto issue_pv = [&](int t, uint32_t v_stage_addr, bool acc, int k_lo, int k_hi, uint32_t a_col) {
         const uint64_t b0 = sw128_desc(v_stage_addr, C::BOX_BYTES, 1024);
 #pragma unroll
         for (int kk = k_lo; kk < k_hi; ++kk) {
-          const uint32_t a = tS(t) + kk * (C::MMA_K * C::EL / 4);
+          const uint32_t a = tS(t) + a_col + kk * (C::MMA_K * C::EL / 4);
           const uint32_t off = (kk * C::MMA_K * 128) >> 4;
           if (FP8)
             mma_f8_ts(tO(t), a, b0 + off, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
@@ -521,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
         const Unit w = get_unit<PAGED>(u, p);
         if (w.nb <= 0) continue;
+        const bool fine0 = tile_fine<FP8>(w, 0, p), fine1 = tile_fine<FP8>(w, 1, p);
         ok = mbar_wait(&sm.q_full[0], nunit & 1, g) && mbar_wait(&sm.q_full[1], nunit & 1, g);
         if (!ok) break;
         // first K block
@@ -573,14 +648,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!ok) break;
             }
             tc_fence_after();
+            const bool fine = t ? fine1 : fine0;
             if (kSplitP) {
-              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, kSplitKeys / C::MMA_K);
+              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, kSplitKeys / C::MMA_K, 0);
+              if (fine) issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, 0, kSplitKeys / C::MMA_K, kFineCol);
               ok = mbar_wait(&sm.p_full[t], pcnt & 1, g);
               if (!ok) break;
               tc_fence_after();
-              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS);
+              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS, 0);
+              if (fine)
+                issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS, kFineCol);
             } else {
-              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, C::PV_KSTEPS);
+              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, C::PV_KSTEPS, 0);
+              if (fine) issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, 0, C::PV_KSTEPS, kFineCol);
             }
             if (!has_next) tc_commit(&sm.o_full[t]);
             if (has_next) {
@@ -629,6 +709,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
       // the MMA multiplies (normalises O so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
+      // fine e4m3 tile: exact running max, P scaled by 2^kFineShift, residual product
+      const bool fine = tile_fine<FP8>(w, t, p);
+      const float thr = fine ? 0.f : kRescaleThreshold;
+      const float shift = fine ? kFineShift : 0.f;
       if (w.nb > 0) {
         int lo, hi;
         key_range(row, w.lk, p, lo, hi);
@@ -659,18 +743,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float mx = fmaxf(max3(pm[0], pm[1], pm[2]), max3(max3(pm[3], pm[4], pm[5]), pm[6], pm[7]));
           const float m_blk = mx * sl2;
           float alpha = 1.f;
-          if (m_blk > m_run + kRescaleThreshold) {
+          if (m_blk > m_run + thr) {
             alpha = ex2_approx(m_run - m_blk);  // m_run = -inf -> 0
             m_run = m_blk;
           }
           l_run *= alpha;
           l_rnd *= alpha;
-          const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+          const float neg_m = (m_run == -INFINITY) ? 0.f : shift - m_run;
           const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
           // P = 2^(s * scale * log2e - m); exact (and rounded) row sums in
           // four independent packed accumulators each.
           uint64_t rs2[4] = {0, 0, 0, 0}, rr2[4] = {0, 0, 0, 0};
-          uint32_t pk[kBN / 2];  // P of the block, packed for the MMA
+          uint32_t pk[kBN / 2];     // P of the block, packed for the MMA
+          uint32_t pk_lo[kBN / 4];  // fine e4m3 tiles: the rounding residual of P
           // Rescale the accumulator when the running max moved.  The previous
           // P.V of this tile has completed: it was issued before this S.
           auto rescale_o = [&]() {
@@ -686,23 +771,27 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           };
+          // P of pairs [Q_LO, Q_HI) into TMEM: bf16 one key pair per column,
+          // e4m3 two pairs (and in fine tiles the residual kFineCol columns on).
+          auto p_part = [&](auto q_lo_c, auto q_hi_c) {
+            constexpr int Q_LO = decltype(q_lo_c)::value, Q_HI = decltype(q_hi_c)::value;
+            constexpr int C0 = FP8 ? Q_LO / 2 : Q_LO, C1 = FP8 ? Q_HI / 2 : Q_HI;
+            if (FP8 && fine) {
+              p_pairs_fine<kRsum, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
+            } else {
+              p_pairs<FP8, kRsum, false, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+              tmem_st_cols<C0, C1>(tS, pk);
+            }
+          };
           if (kSplitP) {
-#pragma unroll
-            for (int q2 = 0; q2 < kSplitKeys / 2; ++q2) p_pair<FP8, kRsum>(q2, sr, sc2, nm2, rs2, rr2, pk);
-            // bf16: one key pair per TMEM column; e4m3: two pairs
-            tmem_st_cols<0, (FP8 ? kSplitKeys / 4 : kSplitKeys / 2)>(tS, pk);
+            p_part(IntC<0>{}, IntC<kSplitKeys / 2>{});
             rescale_o();
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&sm.p_half[t]);
-#pragma unroll
-            for (int q2 = kSplitKeys / 2; q2 < kBN / 2; ++q2) p_pair<FP8, kRsum>(q2, sr, sc2, nm2, rs2, rr2, pk);
-            tmem_st_cols<(FP8 ? kSplitKeys / 4 : kSplitKeys / 2), (FP8 ? kBN / 4 : kBN / 2)>(tS, pk);
+            p_part(IntC<kSplitKeys / 2>{}, IntC<kBN / 2>{});
           } else {
-#pragma unroll
-            for (int q2 = 0; q2 < kBN / 2; ++q2) p_pair<FP8, kRsum>(q2, sr, sc2, nm2, rs2, rr2, pk);
-            tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-            if (!FP8) tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            p_part(IntC<0>{}, IntC<kBN / 2>{});
             rescale_o();
           }
           {
@@ -729,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&sm.st_empty[t], (nunit - 1) & 1, g);
           if (!ok) break;
         }
-        sm.st_m[t][r] = m_run;
+        sm.st_m[t][r] = m_run - shift;  // P carried 2^shift: LSE = m - shift + log2(sum)
         sm.st_l[t][r] = l_run;
         sm.st_r[t][r] = kRsum ? l_rnd : l_run;
         mbar_arrive(&sm.st_full[t]);

@@ -55,6 +55,10 @@
  *     bounds-check mode) are recorded in the device status word and reported
  *     by attn_last_device_error().  The kernels never trap.
  *   - Tensors are contiguous, row-major, with a 16-byte aligned base.
+ *   - Per-device state (the status word's address, kernel attributes) is
+ *     looked up on first use on each device and cached for the life of the
+ *     process; after cudaDeviceReset the library must not be used again in
+ *     that process.
  */
 #ifndef ATTN_SM100_H
 #define ATTN_SM100_H
@@ -297,15 +301,24 @@ ATTN_API int attn_kv_append(const void* k_new, const void* v_new, void* k_pages,
  * the library until the process exits), so the call allocates nothing:
  * no cudaMalloc, cudaFree or allocating library routine.
  *
- * Arguments, layouts, supported sizes and results are those of
- * attn_decode_paged, without the workspace.  Sizes whose scratch
- * (attn_decode_workspace_bytes) exceeds the array return ATTN_ERR_INVALID
- * before anything is launched, with the sizes in attn_last_error_message().
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the one array and it keeps the previous call's
- * contents (nothing in it needs to start at zero); calls that overlap on the
- * GPU -- different streams with no ordering between them -- race on it.
+ * Arguments, layouts, supported sizes, argument checks and results are those
+ * of attn_decode_paged, without the workspace.  Sizes that pass those checks
+ * but whose scratch (attn_decode_workspace_bytes) exceeds the array return
+ * ATTN_ERR_INVALID before anything is launched, with the sizes in
+ * attn_last_error_message().
+ * Set-up: the CUDA runtime loads the array onto a GPU when it is first needed
+ * there -- under lazy module loading (the default), at the first call of this
+ * entry point on that device, which looks up the array's address.  That first
+ * call per device therefore allocates the array and may synchronise: make it
+ * once at start-up, with the device current, outside any context that forbids
+ * allocation or synchronisation and before any stream capture (a call with
+ * B == 0 does only this set-up).  Later calls on that device allocate nothing.
+ * All calls share the one array and it keeps the previous call's contents
+ * (nothing in it needs to start at zero); calls that overlap on the GPU --
+ * different streams with no ordering between them -- race on it.  The array's
+ * address is cached per device for the process: after cudaDeviceReset this
+ * library (which caches its other per-device state the same way) must not be
+ * used again in that process.
  */
 #define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
 ATTN_API int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,

@@ -57,6 +57,43 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, which):
         assert do <= O_TOL and dl <= LSE_TOL, (do, dl)
 
 
+def test_noalloc_call_allocates_no_device_memory(lib):
+    """After the set-up call (the first on the device, here with B = 0, which
+    loads the array), a decode call leaves the device's free memory and the
+    caching allocator's counters unchanged."""
+    cdll = lib.load()
+    shape = DecodeShape("alloc", B=8, Hq=32, Hkv=1, D=128, len_lo=100, len_hi=3000)
+    kv = decode_inputs(shape, 18)
+    d = {n: getattr(kv, n).cuda() for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+    o = torch.empty_like(d["q"])
+    lse = torch.empty(d["q"].shape[:2], dtype=torch.float32, device="cuda")
+    setup = DecodeShape("setup", B=0, Hq=32, Hkv=1, D=128, len_lo=1, len_hi=1)
+    assert _noalloc_call(cdll, d, setup, o, lse) == 0
+    assert _noalloc_call(cdll, d, shape, o, lse) == 0      # first real call: kernels loaded
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    stats0 = torch.cuda.memory_stats()
+    assert _noalloc_call(cdll, d, shape, o, lse) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    stats1 = torch.cuda.memory_stats()
+    assert lib.attn_last_device_error() == 0
+    assert free1 == free0
+    for key in ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
+
+
+def test_noalloc_checks_arguments_like_the_workspace_entry_point(lib):
+    """An unsupported shape is refused as attn_decode_paged refuses it, even
+    when its scratch would also be too large for the array."""
+    cdll = lib.load()
+    fake = ctypes.c_void_p(0x10000)
+    B, Hq, D, max_pages = 256, 64, 96, 4096         # D = 96: not built
+    st = cdll.attn_decode_paged_noalloc(fake, fake, fake, fake, fake, fake, fake, B, Hq, 1, D, 16, 10,
+                                        max_pages, ctypes.c_float(0.1), ctypes.c_void_p(0))
+    assert st == lib.ATTN_ERR_UNSUPPORTED
+
+
 def test_noalloc_rejects_sizes_beyond_its_array(lib):
     cdll = lib.load()
     limit = 32 << 20
@@ -66,4 +103,5 @@ def test_noalloc_rejects_sizes_beyond_its_array(lib):
     st = cdll.attn_decode_paged_noalloc(fake, fake, fake, fake, fake, fake, fake, B, Hq, 1, D, 16, 10,
                                         max_pages, ctypes.c_float(0.1), ctypes.c_void_p(0))
     assert st == lib.ATTN_ERR_INVALID
-    assert "scratch" in lib.attn_last_error_message()
+    msg = lib.attn_last_error_message()
+    assert "scratch" in msg and "invalid argument" not in msg
