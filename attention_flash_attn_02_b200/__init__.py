@@ -60,6 +60,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_fwd.restype = c_int
     lib.attn_fwd_fp8.argtypes = [c_void_p] * 5 + [c_int] * 6 + [c_float, c_int, c_int] + [c_float] * 3 + [c_void_p]
     lib.attn_fwd_fp8.restype = c_int
+    lib.attn_fwd_e5m2.argtypes = lib.attn_fwd_fp8.argtypes
+    lib.attn_fwd_e5m2.restype = c_int
     lib.attn_decode_workspace_bytes.argtypes = [c_int] * 4
     lib.attn_decode_workspace_bytes.restype = c_size_t
     lib.attn_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p, c_size_t, c_void_p]
@@ -138,6 +140,20 @@ def attn_fwd_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float,
                  scale: Optional[float] = None, causal: bool = False, window: int = 0,
                  o=None, lse=None, stream=None):
     """e4m3 attention forward (bf16 output); tensors torch.float8_e4m3fn."""
+    return _fwd_8bit("attn_fwd_fp8", "float8_e4m3fn", q, k, v, q_descale, k_descale, v_descale, scale, causal,
+                     window, o, lse, stream)
+
+
+def attn_fwd_e5m2(q, k, v, q_descale: float, k_descale: float, v_descale: float,
+                  scale: Optional[float] = None, causal: bool = False, window: int = 0,
+                  o=None, lse=None, stream=None):
+    """e5m2 attention forward (bf16 output); tensors torch.float8_e5m2."""
+    return _fwd_8bit("attn_fwd_e5m2", "float8_e5m2", q, k, v, q_descale, k_descale, v_descale, scale, causal,
+                     window, o, lse, stream)
+
+
+def _fwd_8bit(name, dtype_name, q, k, v, q_descale, k_descale, v_descale, scale, causal, window, o, lse,
+              stream):
     import torch
     lib = load()
     B, Hq, Lq, D = q.shape
@@ -149,12 +165,12 @@ def attn_fwd_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float,
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
     for t in (q, k, v):
-        if t.dtype != torch.float8_e4m3fn or not t.is_contiguous():
-            raise TypeError("attn_fwd_fp8: q, k, v must be contiguous float8_e4m3fn")
-    st = lib.attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
-                          float(scale), int(bool(causal)), int(window), float(q_descale),
-                          float(k_descale), float(v_descale), _stream_handle(stream))
-    _check(st, "attn_fwd_fp8")
+        if t.dtype != getattr(torch, dtype_name) or not t.is_contiguous():
+            raise TypeError(f"{name}: q, k, v must be contiguous {dtype_name}")
+    st = getattr(lib, name)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
+                            float(scale), int(bool(causal)), int(window), float(q_descale),
+                            float(k_descale), float(v_descale), _stream_handle(stream))
+    _check(st, name)
     return o, lse
 
 

@@ -114,6 +114,20 @@ ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
   return launch_prefill(a, static_cast<cudaStream_t>(stream));
 }
 
+ATTN_API int attn_fwd_e5m2(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                           int Hkv, int Lq, int Lk, int D, float scale, int causal, int window, float q_descale,
+                           float k_descale, float v_descale, attn_stream_t stream) {
+  int st = validate_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (!(q_descale > 0.f) || !(k_descale > 0.f) || !(v_descale > 0.f)) return ATTN_ERR_INVALID;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * Lq == 0) return ATTN_OK;
+  PrefillArgs a{q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, window > 0 ? window : 0, true,
+                q_descale, k_descale, v_descale};
+  a.e5m2 = true;
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D) {
   if (B <= 0 || Hq <= 0 || max_pages_per_seq <= 0 || D <= 0) return 0;
   return decode_workspace_bytes(B, Hq, max_pages_per_seq, D);

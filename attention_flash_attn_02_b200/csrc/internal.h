@@ -25,6 +25,7 @@ struct PrefillArgs {
   const int* block_table;
   const int* seq_lens;
   int num_pages, max_pages;
+  bool e5m2 = false;  // fp8 inputs in e5m2 (else e4m3)
 };
 
 struct DecodeArgs {

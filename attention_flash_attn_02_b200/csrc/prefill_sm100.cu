@@ -104,7 +104,9 @@ static_assert(ATTN_SPLIT_P == 0 || (ATTN_SPLIT_P % 2 == 0 && ATTN_SPLIT_P < 8), 
 #endif
 static_assert(ATTN_ROUNDED_SUM == 0 || ATTN_ROUNDED_SUM == 1, "row-sum mode 0 or 1");
 
-template <int D, bool FP8>
+// E5M2 (with FP8): the 8-bit inputs are e5m2, and P is multiplied in e5m2 too
+// (kind::f8f6f4 format code 1; each product keeps one operand type).
+template <int D, bool FP8, bool E5M2 = false>
 struct Cfg {
   static constexpr int EL = FP8 ? 1 : 2;                 // bytes per element
   static constexpr int ROW_BYTES = D * EL;
@@ -121,8 +123,9 @@ struct Cfg {
   static constexpr int S_KSTEPS = D / MMA_K;
   static constexpr int PV_KSTEPS = kBN / MMA_K;
   static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
-  static constexpr uint32_t IDESC_S = make_idesc(FP8 ? 0u : 1u, kBM, kBN, false);
-  static constexpr uint32_t IDESC_PV = make_idesc(FP8 ? 0u : 1u, kBM, D, true);
+  static constexpr uint32_t FMT = FP8 ? (E5M2 ? 1u : 0u) : 1u;  // e4m3 0, e5m2 1; bf16 1
+  static constexpr uint32_t IDESC_S = make_idesc(FMT, kBM, kBN, false);
+  static constexpr uint32_t IDESC_PV = make_idesc(FMT, kBM, D, true);
   // shared memory: [Q0][Q1][stage 0..NS-1] (1024-aligned) + barriers
   static constexpr int SMEM_TILES = (2 + NS) * TILE_BYTES;
   static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align slack*/ + 4096 /*barriers, row statistics*/;
@@ -143,6 +146,7 @@ struct Params {
   int causal, window;
   float scale_log2;  // logit scale * log2(e) (fp8: times both descales)
   float out_scale;   // 1 (bf16) or v_descale (fp8)
+
   int* status;
   unsigned long long timeout_ns;
   int stall;  // testing hook: the producer issues no loads, every wait runs out
@@ -275,9 +279,10 @@ static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserv
 // ex2, or for kEmuPairsPer8 of every 8 pairs the FMA-pipe polynomial), packed
 // for the MMA, added to the exact row sum and, with RSUM, to the sum of the
 // rounded values.  e4m3 pairs go two to a 32-bit word.
-// FINE (e4m3 only): also the residual e4m3(P - h) into pk_lo, and the sum of
-// h + residual, the weight the two products apply together.
-template <bool FP8, bool RSUM, bool FINE>
+// FINE (8-bit P only): also the residual fp8(P - h) into pk_lo, and the sum
+// of h + residual, the weight the two products apply together.  E5M2: P and
+// its residual in e5m2 (the format of e5m2 inputs), else e4m3.
+template <bool FP8, bool RSUM, bool FINE, bool E5M2 = false>
 __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
                                        uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
                                        uint32_t (&pk_lo)[kBN / 4]) {
@@ -293,26 +298,18 @@ __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64
   }
   rs2[q2 & 3] = add2(rs2[q2 & 3], f2(p0, p1));
   if (FP8) {
-    const uint16_t e = pack_e4m3x2(p0, p1);
+    const uint16_t e = E5M2 ? pack_e5m2x2(p0, p1) : pack_e4m3x2(p0, p1);
     if (q2 & 1) pk[q2 >> 1] |= (uint32_t)e << 16;
     else pk[q2 >> 1] = e;
-    uint32_t h;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(e));
     float h0, h1;
-    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-        : "=f"(h0), "=f"(h1)
-        : "r"(h));
+    unpack_fp8x2<E5M2>(e, h0, h1);
     if (FINE) {
-      // P - h is exact in fp32 (h is P rounded to a 4-bit significand).
-      const uint16_t el = pack_e4m3x2(p0 - h0, p1 - h1);
+      // P - h is exact in fp32 (h is P rounded to a 3- or 4-bit significand).
+      const uint16_t el = E5M2 ? pack_e5m2x2(p0 - h0, p1 - h1) : pack_e4m3x2(p0 - h0, p1 - h1);
       if (q2 & 1) pk_lo[q2 >> 1] |= (uint32_t)el << 16;
       else pk_lo[q2 >> 1] = el;
-      uint32_t hl;
-      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hl) : "h"(el));
       float l0, l1;
-      asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-          : "=f"(l0), "=f"(l1)
-          : "r"(hl));
+      unpack_fp8x2<E5M2>(el, l0, l1);
       h0 += l0;
       h1 += l1;
     }
@@ -324,33 +321,34 @@ __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64
   }
 }
 
-template <bool FP8, bool RSUM, bool FINE, int Q_LO, int Q_HI>
+template <bool FP8, bool RSUM, bool FINE, int Q_LO, int Q_HI, bool E5M2 = false>
 __device__ __forceinline__ void p_pairs(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2, uint64_t (&rs2)[4],
                                         uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2], uint32_t (&pk_lo)[kBN / 4]) {
 #pragma unroll
-  for (int q2 = Q_LO; q2 < Q_HI; ++q2) p_pair<FP8, RSUM, FINE>(q2, sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+  for (int q2 = Q_LO; q2 < Q_HI; ++q2) p_pair<FP8, RSUM, FINE, E5M2>(q2, sr, sc2, nm2, rs2, rr2, pk, pk_lo);
 }
 
 // Fine e4m3 tiles: pairs [Q_LO, Q_HI) in chunks of 16 (32 keys), each chunk's
 // P and residual stored to TMEM at once (columns Q/2 on, at taddr and
 // taddr + kFineCol), so that the residual adds few live registers.
-template <bool RSUM, int Q_LO, int Q_HI>
+template <bool RSUM, bool E5M2, int Q_LO, int Q_HI>
 __device__ __forceinline__ void p_pairs_fine(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
                                              uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
                                              uint32_t (&pk_lo)[kBN / 4], uint32_t taddr) {
   if constexpr (Q_LO < Q_HI) {
     constexpr int QE = Q_LO + 16 < Q_HI ? Q_LO + 16 : Q_HI;
-    p_pairs<true, RSUM, true, Q_LO, QE>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+    p_pairs<true, RSUM, true, Q_LO, QE, E5M2>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
     tmem_st_cols<Q_LO / 2, QE / 2>(taddr, pk);
     tmem_st_cols<Q_LO / 2, QE / 2>(taddr + kFineCol, pk_lo);
-    p_pairs_fine<RSUM, QE, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, taddr);
+    p_pairs_fine<RSUM, E5M2, QE, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, taddr);
   }
 }
 
 // Is tile t of unit w a "fine" e4m3 tile (its first row sees < kFineKeys keys)?
-template <bool FP8>
+template <bool FP8, bool E5M2>
 __device__ __forceinline__ bool tile_fine(const Unit& w, int t, const Params& p) {
   if (!FP8) return false;
+  if (E5M2) return true;  // 2 mantissa bits: every tile takes the residual product
   const int m0 = w.m0_of(t);
   if (m0 >= p.Lq) return false;
   int lo, hi;
@@ -358,11 +356,11 @@ __device__ __forceinline__ bool tile_fine(const Unit& w, int t, const Params& p)
   return hi - lo < kFineKeys;
 }
 
-template <int D, bool FP8, bool PAGED>
+template <int D, bool FP8, bool PAGED, bool E5M2>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  using C = Cfg<D, FP8>;
+  using C = Cfg<D, FP8, E5M2>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t tiles_addr = (raw_addr + 1023u) & ~1023u;
@@ -595,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
         const Unit w = get_unit<PAGED>(u, p);
         if (w.nb <= 0) continue;
-        const bool fine0 = tile_fine<FP8>(w, 0, p), fine1 = tile_fine<FP8>(w, 1, p);
+        const bool fine0 = tile_fine<FP8, E5M2>(w, 0, p), fine1 = tile_fine<FP8, E5M2>(w, 1, p);
         ok = mbar_wait(&sm.q_full[0], nunit & 1, g) && mbar_wait(&sm.q_full[1], nunit & 1, g);
         if (!ok) break;
         // first K block
@@ -710,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the MMA multiplies (normalises O so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
       // fine e4m3 tile: exact running max, P scaled by 2^kFineShift, residual product
-      const bool fine = tile_fine<FP8>(w, t, p);
+      const bool fine = tile_fine<FP8, E5M2>(w, t, p);
       const float thr = fine ? 0.f : kRescaleThreshold;
       const float shift = fine ? kFineShift : 0.f;
       if (w.nb > 0) {
@@ -776,8 +774,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           auto p_part = [&](auto q_lo_c, auto q_hi_c) {
             constexpr int Q_LO = decltype(q_lo_c)::value, Q_HI = decltype(q_hi_c)::value;
             constexpr int C0 = FP8 ? Q_LO / 2 : Q_LO, C1 = FP8 ? Q_HI / 2 : Q_HI;
-            if (FP8 && fine) {
-              p_pairs_fine<kRsum, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
+            if (FP8 && (E5M2 || fine)) {
+              p_pairs_fine<kRsum, E5M2, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
             } else {
               p_pairs<FP8, kRsum, false, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
               tmem_st_cols<C0, C1>(tS, pk);
@@ -873,15 +871,15 @@ bool encode_pool(CUtensorMap* map, const void* pool, bool fp8, int D, int num_pa
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, bool PAGED>
+template <int D, bool FP8, bool PAGED, bool E5M2 = false>
 int run(const PrefillArgs& a, cudaStream_t stream) {
-  using C = Cfg<D, FP8>;
+  using C = Cfg<D, FP8, E5M2>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
   if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(prefill_kernel<D, FP8, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(prefill_kernel<D, FP8, PAGED, E5M2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_BYTES);
     if (err != cudaSuccess) return fail_cuda("prefill: cudaFuncSetAttribute", err);
     attr_set[dev] = true;
@@ -909,6 +907,7 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   const float log2e = 1.4426950408889634f;
   p.scale_log2 = a.scale * log2e * (FP8 ? a.q_descale * a.k_descale : 1.f);
   p.out_scale = FP8 ? a.v_descale : 1.f;
+
   p.status = device_status_word();
   if (!p.status) return fail_cuda("prefill: status word", cudaGetLastError());
   p.timeout_ns = wait_timeout_ns();
@@ -925,7 +924,7 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
     if (!encode_pool(&tk, a.k, FP8, D, a.num_pages, a.Hkv) || !encode_pool(&tv, a.v, FP8, D, a.num_pages, a.Hkv))
       return fail_cuda("prefill: tensor map (pool)", cudaErrorInvalidValue);
     const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
-    prefill_kernel<D, FP8, PAGED><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    prefill_kernel<D, FP8, PAGED, E5M2><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     err = cudaGetLastError();
     return err == cudaSuccess ? 0 : fail_cuda("prefill (paged): launch", err);
   }
@@ -937,7 +936,7 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   if (!encode_3d(&tv, have_k ? a.v : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
     return fail_cuda("prefill: tensor map (v)", cudaErrorInvalidValue);
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
-  prefill_kernel<D, FP8, PAGED><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, FP8, PAGED, E5M2><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   err = cudaGetLastError();
   return err == cudaSuccess ? 0 : fail_cuda("prefill: launch", err);
 }
@@ -952,8 +951,8 @@ int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     return -2;
   }
   if (a.fp8) {
-    if (a.D == 128) return run<128, true, false>(a, stream);
-    return -2;
+    if (a.D != 128) return -2;
+    return a.e5m2 ? run<128, true, false, true>(a, stream) : run<128, true, false>(a, stream);
   }
   if (a.D == 128) return run<128, false, false>(a, stream);
   if (a.D == 64) return run<64, false, false>(a, stream);

@@ -418,6 +418,25 @@ __device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Two floats -> packed e5m2x2 (lo in bits 0..7), round to nearest even, saturating.
+__device__ __forceinline__ uint16_t pack_e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Packed fp8x2 (e4m3 or e5m2) -> the two values in fp32 (exact: via f16).
+template <bool E5M2>
+__device__ __forceinline__ void unpack_fp8x2(uint16_t v, float& lo, float& hi) {
+  uint32_t h;
+  if (E5M2)
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(v));
+  else
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+}
+
 // Sum of the two bf16 halves of a packed pair, in fp32 (exact conversion).
 __device__ __forceinline__ float sum_bf16x2(uint32_t v) {
   return __uint_as_float(v << 16) + __uint_as_float(v & 0xFFFF0000u);

@@ -4,7 +4,8 @@
  *
  * Operations, all on one GPU:
  *
- *   attn_fwd / attn_fwd_fp8   fused, tiled scaled-dot-product attention
+ *   attn_fwd / attn_fwd_fp8 / attn_fwd_e5m2
+ *                             fused, tiled scaled-dot-product attention
  *                             O = softmax(scale * Q K^T + mask) V, with the
  *                             per-row log-sum-exp, computed with the online
  *                             softmax recurrence (running row max and sum,
@@ -34,7 +35,7 @@
  *     h % g == 0), §4.1-4.2 (tiling into SRAM, online softmax, one fused
  *     kernel).
  *   - "注意力机制深度优化" (kler.cn) §一.1 (FP8 e4m3), §一.2 (skipping the
- *     upper-right causal triangle).
+ *     upper-right causal triangle), §四.2 (FP8 e5m2).
  *
  * Conventions shared by every entry point
  *   - Pointers are DEVICE pointers unless stated otherwise.  The caller owns
@@ -135,6 +136,26 @@ ATTN_API int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
                           float scale, int causal, int window,
                           float q_descale, float k_descale, float v_descale,
                           attn_stream_t stream);
+
+/*
+ * attn_fwd_e5m2 -- attn_fwd_fp8 on float8_e5m2 inputs (the e5m2 FP8 format of
+ * the kler.cn page §四.2, "torch_dtype=torch.float8_e5m2"), bf16 output.
+ *
+ *   q, k, v  e5m2 bytes, same shapes/layout as attn_fwd; o bf16; lse fp32.
+ *   q_descale, k_descale, v_descale: per-tensor scales as attn_fwd_fp8.
+ * The logits come from an e5m2 x e5m2 product with fp32 accumulation.  The
+ * weights P (fp32 softmax, scaled by 2^8 with an exact running max) are
+ * multiplied with V in e5m2 -- one operand type per product -- as two terms,
+ * e5m2(P) and the e5m2 rounding residual of P, so each weight carries about 6
+ * significant bits (e5m2 alone has 3); O is multiplied by v_descale.
+ *
+ * Supported: D == 128 only (ATTN_ERR_UNSUPPORTED otherwise).
+ */
+ATTN_API int attn_fwd_e5m2(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                           float scale, int causal, int window,
+                           float q_descale, float k_descale, float v_descale,
+                           attn_stream_t stream);
 
 /*
  * attn_bwd_workspace_bytes -- scratch attn_bwd needs: an fp32 dQ accumulator

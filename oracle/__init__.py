@@ -30,6 +30,7 @@ from .sdpa import (  # noqa: F401
     attention_backward,
     attention_fp8,
     dequantize_e4m3,
+    dequantize_e5m2,
     gather_pages,
     kv_cache_bytes,
     merge_partials,

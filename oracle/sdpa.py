@@ -140,6 +140,14 @@ def dequantize_e4m3(x8, s: float) -> np.ndarray:
     return _f64(x8) * float(s)
 
 
+def dequantize_e5m2(x8, s: float) -> np.ndarray:
+    """Value of a per-tensor scaled e5m2 tensor: float64(x8) * s (the
+    ``torch_dtype=torch.float8_e5m2`` format named in p1 §四.2).  Both 8-bit
+    formats convert exactly to float64; the two functions differ only in the
+    format they are pinned against."""
+    return _f64(x8) * float(s)
+
+
 def attention_backward(q, k, v, o, do, lse, scale: float, causal: bool = False, window: int = 0):
     """Gradients of O = softmax(scale * Q K^T + mask) V with respect to Q, K
     and V, in float64, from the forward's O and per-row LSE.
@@ -189,11 +197,12 @@ def attention_backward(q, k, v, o, do, lse, scale: float, causal: bool = False, 
 
 def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale: float,
                   causal: bool = False, window: int = 0, **kw):
-    """Attention on e4m3 inputs: the plain definition applied to the exact
-    dequantised values, so the oracle measures kernel error and not
-    quantisation error."""
-    return attention(dequantize_e4m3(q8, q_scale), dequantize_e4m3(k8, k_scale),
-                     dequantize_e4m3(v8, v_scale), scale, causal, window, **kw)
+    """Attention on 8-bit inputs (e4m3 or e5m2, per-tensor scales): the plain
+    definition applied to the exact dequantised values, so the oracle
+    measures kernel error and not quantisation error."""
+    deq = dequantize_e5m2 if (torch is not None and isinstance(q8, torch.Tensor)
+                              and q8.dtype == torch.float8_e5m2) else dequantize_e4m3
+    return attention(deq(q8, q_scale), deq(k8, k_scale), deq(v8, v_scale), scale, causal, window, **kw)
 
 
 def online_softmax_attention(q, k, v, scale: float, causal: bool = False, window: int = 0,

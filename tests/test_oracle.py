@@ -550,6 +550,28 @@ def test_fp8_attention_is_definition_on_dequantised_values():
     assert abs(float((q8.float().abs().max()))) == 448.0
 
 
+def test_e5m2_dequantisation_known_codes():
+    """OCP FP8 e5m2 (float8_e5m2, 5 exponent bits with bias 15, 2 mantissa
+    bits): 0x3C = 1.0, 0x7B = 1.75 * 2^15 = 57344 (max finite), 0x01 =
+    2^-16 (smallest subnormal), 0xC0 = -2.0."""
+    codes = torch.tensor([0x3C, 0x7B, 0x01, 0xC0], dtype=torch.uint8).view(torch.float8_e5m2)
+    vals = oracle.dequantize_e5m2(codes, 0.5)
+    np.testing.assert_array_equal(vals, [0.5, 28672.0, 2.0 ** -17, -1.0])
+
+
+def test_e5m2_attention_is_definition_on_dequantised_values():
+    shape = PrefillShape("t", B=1, Hq=2, Hkv=1, Lq=7, Lk=11, D=4, causal=True, fp8=True)
+    q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, 4, fmt="e5m2")
+    assert q8.dtype == torch.float8_e5m2
+    o, lse = oracle.attention_fp8(q8, k8, v8, sq, sk, sv, 0.5, causal=True, window=3)
+    ob, lb = _brute((q8.double() * sq).numpy(), (k8.double() * sk).numpy(), (v8.double() * sv).numpy(),
+                    0.5, True, 3)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lb, rtol=0, atol=1e-13)
+    # quantisation scale: amax maps to the largest finite e5m2 value
+    assert float(q8.float().abs().max()) == 57344.0
+
+
 def test_tiny_workload_golden_rows():
     """Regression fixture written by tests/golden/make_golden.py (which
     calls only the oracle): selected rows of the tiny MHA workload."""

@@ -199,6 +199,49 @@ def test_fp8_full_size_rows(lib):
     _check(o[0][heads][:, rows], o_ref[0], lse[0][heads][:, rows], l_ref[0], FP8_TOL, what=shape.name)
 
 
+E5M2_SWEEP = [
+    (1, 4, 2, 1100, 1100, True, 0),
+    (1, 3, 3, 300, 300, True, 2),       # rows of two keys
+    (1, 4, 2, 700, 700, True, 300),
+    (1, 4, 4, 100, 900, True, 0),       # Lq < Lk
+    (1, 2, 2, 300, 100, True, 0),       # Lq > Lk: first rows see no key
+    (2, 2, 1, 77, 200, False, 0),
+]
+
+
+def _run_e5m2(lib, shape, seed):
+    q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, seed, fmt="e5m2")
+    o, lse = lib.attn_fwd_e5m2(q8.cuda(), k8.cuda(), v8.cuda(), sq, sk, sv, shape.scale, shape.causal,
+                               shape.window)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    return (q8, k8, v8, sq, sk, sv), o, lse
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,causal,window", E5M2_SWEEP)
+def test_e5m2_sweep(lib, B, Hq, Hkv, Lq, Lk, causal, window):
+    """float8_e5m2 inputs (kler.cn §四.2): e5m2 products, P multiplied with V
+    as e5m2 and its e5m2 residual; the FP8 bound."""
+    shape = PrefillShape("e5m2", B, Hq, Hkv, Lq, Lk, 128, causal, window=window, fp8=True)
+    ins, o, lse = _run_e5m2(lib, shape, 17 + Lq + Lk + window)
+    o_ref, l_ref = oracle.attention_fp8(*ins, shape.scale, causal, window)
+    _check(o, o_ref, lse, l_ref, FP8_TOL, what=f"e5m2 {shape}")
+
+
+def test_e5m2_full_size_rows(lib):
+    """The long-context FP8 workload's shape (B1 Hq32 L32768, causal) with
+    e5m2 inputs: rows 0..127 of all heads and sampled rows of three heads."""
+    shape = FP8_CAUSAL
+    ins, o, lse = _run_e5m2(lib, shape, seed_of(4))
+    first = list(range(128))
+    o_ref, l_ref = oracle.attention_fp8(*ins, shape.scale, True, rows=first, batches=[0])
+    _check(o[0][:, first], o_ref[0], lse[0][:, first], l_ref[0], FP8_TOL, what="e5m2 rows 0-127")
+    rows = _sampled_rows(shape.Lq, 12, 5)
+    heads = [2, 17, 30]
+    o_ref, l_ref = oracle.attention_fp8(*ins, shape.scale, True, rows=rows, heads=heads, batches=[0])
+    _check(o[0][heads][:, rows], o_ref[0], lse[0][heads][:, rows], l_ref[0], FP8_TOL, what="e5m2 sampled")
+
+
 def _whole_heads(q, k, v, shape, b, heads, o, lse, tol=BF16_TOL, chunk=2048):
     """Every row of the given heads of batch b against the oracle, in row
     chunks (each chunk's score block spans only its visible keys)."""

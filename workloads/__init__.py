@@ -16,6 +16,8 @@ Recipe (one ``torch.Generator`` per call, seeded by the caller):
   value), ``x8 = cast(x / s)``.  This is the input preparation of the
   long-context FP8 workload; the kernel and the oracle both receive ``x8`` and
   ``s``.
+* FP8 e5m2 prefill: the same draws quantised to ``float8_e5m2`` with
+  ``s = amax(|x|) / 57344`` (the largest finite e5m2 value).
 * paged decode: q ``[B, Hq, D]``, then per-sequence lengths uniform in
   ``[len_lo, len_hi]`` (so that the pool can be sized from them), then the K
   pool, then the V pool (pools are ``[num_pages, page_size, Hkv, D]``), then a
@@ -31,6 +33,7 @@ from typing import Optional
 import torch
 
 FP8_E4M3_MAX = 448.0
+FP8_E5M2_MAX = 57344.0
 PAGE_SIZE = 16
 
 
@@ -114,15 +117,28 @@ def quantize_e4m3(x: torch.Tensor):
     return x8, float(scale)
 
 
-def prefill_inputs_fp8(shape: PrefillShape, seed: int):
-    """(q8, k8, v8, q_scale, k_scale, v_scale); tensors float8_e4m3fn [B, H, L, D]."""
+def quantize_e5m2(x: torch.Tensor):
+    """Per-tensor e5m2 quantisation of an fp32 tensor: (x8, scale), with
+    ``scale = amax/57344`` (the largest finite e5m2 value) and torch's
+    round-to-nearest-even cast to ``float8_e5m2``."""
+    amax = x.abs().max().to(torch.float32)
+    scale = (amax / FP8_E5M2_MAX).item() if amax > 0 else 1.0
+    x8 = (x / scale).to(torch.float8_e5m2)
+    return x8, float(scale)
+
+
+def prefill_inputs_fp8(shape: PrefillShape, seed: int, fmt: str = "e4m3"):
+    """(q8, k8, v8, q_scale, k_scale, v_scale); tensors float8_e4m3fn (or,
+    with ``fmt="e5m2"``, float8_e5m2) [B, H, L, D], from the same fp32 draws
+    as ``prefill_inputs``."""
     g = _gen(seed)
     q = _normal(g, (shape.B, shape.Hq, shape.Lq, shape.D))
     k = _normal(g, (shape.B, shape.Hkv, shape.Lk, shape.D))
     v = _normal(g, (shape.B, shape.Hkv, shape.Lk, shape.D))
-    q8, sq = quantize_e4m3(q)
-    k8, sk = quantize_e4m3(k)
-    v8, sv = quantize_e4m3(v)
+    quant = {"e4m3": quantize_e4m3, "e5m2": quantize_e5m2}[fmt]
+    q8, sq = quant(q)
+    k8, sk = quant(k)
+    v8, sv = quant(v)
     return q8, k8, v8, sq, sk, sv
 
 
