@@ -62,6 +62,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_fwd_fp8.restype = c_int
     lib.attn_fwd_e5m2.argtypes = lib.attn_fwd_fp8.argtypes
     lib.attn_fwd_e5m2.restype = c_int
+    lib.attn_fwd_mla.argtypes = [c_void_p] * 5 + [c_int] * 7 + [c_float, c_int, c_int, c_void_p]
+    lib.attn_fwd_mla.restype = c_int
     lib.attn_decode_workspace_bytes.argtypes = [c_int] * 4
     lib.attn_decode_workspace_bytes.restype = c_size_t
     lib.attn_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_void_p, c_size_t, c_void_p]
@@ -133,6 +135,33 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, windo
     st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
                       float(scale), int(bool(causal)), int(window), _stream_handle(stream))
     _check(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_mla(q, k, v, scale: Optional[float] = None, causal: bool = False, window: int = 0,
+                 o=None, lse=None, stream=None):
+    """bf16 attention with query/key width D_qk and value width D_v (each 64,
+    128, 192 or 256): q [B, Hq, Lq, D_qk], k [B, Hkv, Lk, D_qk], v [B, Hkv, Lk,
+    D_v]; returns (o [B, Hq, Lq, D_v] bf16, lse [B, Hq, Lq] fp32).  The default
+    scale is 1/sqrt(D_qk)."""
+    import torch
+    lib = load()
+    B, Hq, Lq, Dqk = q.shape
+    Hkv, Lk, Dv = k.shape[1], k.shape[2], v.shape[3]
+    if k.shape[3] != Dqk or v.shape[:3] != k.shape[:3]:
+        raise ValueError("attn_fwd_mla: k must be [B, Hkv, Lk, D_qk] and v [B, Hkv, Lk, D_v]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dqk)
+    if o is None:
+        o = torch.empty((B, Hq, Lq, Dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise TypeError("attn_fwd_mla: q, k, v must be contiguous bfloat16")
+    st = lib.attn_fwd_mla(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, Dqk, Dv,
+                          float(scale), int(bool(causal)), int(window), _stream_handle(stream))
+    _check(st, "attn_fwd_mla")
     return o, lse
 
 

@@ -128,6 +128,19 @@ ATTN_API int attn_fwd_e5m2(const void* q, const void* k, const void* v, void* o,
   return launch_prefill(a, static_cast<cudaStream_t>(stream));
 }
 
+ATTN_API int attn_fwd_mla(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                          int Hkv, int Lq, int Lk, int D_qk, int D_v, float scale, int causal, int window,
+                          attn_stream_t stream) {
+  if (D_v <= 0) return ATTN_ERR_INVALID;
+  int st = validate_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D_qk, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  auto ok_dim = [](int d) { return d == 64 || d == 128 || d == 192 || d == 256; };
+  if (!ok_dim(D_qk) || !ok_dim(D_v)) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * Lq == 0) return ATTN_OK;
+  WideArgs a{q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D_qk, D_v, scale, causal, window > 0 ? window : 0};
+  return launch_prefill_wide(a, static_cast<cudaStream_t>(stream));
+}
+
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D) {
   if (B <= 0 || Hq <= 0 || max_pages_per_seq <= 0 || D <= 0) return 0;
   return decode_workspace_bytes(B, Hq, max_pages_per_seq, D);

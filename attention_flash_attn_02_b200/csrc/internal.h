@@ -28,6 +28,19 @@ struct PrefillArgs {
   bool e5m2 = false;  // fp8 inputs in e5m2 (else e4m3)
 };
 
+// Attention with query/key width Dqk and value width Dv (64..256 each).
+struct WideArgs {
+  const void* q;  // [B, Hq, Lq, Dqk] bf16
+  const void* k;  // [B, Hkv, Lk, Dqk]
+  const void* v;  // [B, Hkv, Lk, Dv]
+  void* o;        // [B, Hq, Lq, Dv]
+  float* lse;
+  int B, Hq, Hkv, Lq, Lk, Dqk, Dv;
+  float scale;
+  int causal, window;
+};
+int launch_prefill_wide(const WideArgs& a, cudaStream_t stream);
+
 struct DecodeArgs {
   const void* q;
   const void* k_pages;

@@ -74,7 +74,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // columns [0, 32); all 128 columns of S are in registers by then).
 constexpr int kFineKeys = 512;
 constexpr float kFineShift = 8.0f;
-constexpr uint32_t kFineCol = 32;
+// bf16 tiles take the same two-part product (bf16(P) and bf16(P - bf16(P)),
+// the residual in columns [64, 128)) when their first row sees fewer than
+// kFineKeysBf16 keys: rounding P to bf16 moves the O of a row of two keys by
+// up to ~2^-9 of the spread of its V values, which with the bf16 rounding of O
+// can pass 1e-2.  bf16 needs no scaling (its exponent range is fp32's).
+constexpr int kFineKeysBf16 = 256;
+template <bool FP8>
+constexpr uint32_t kFineCol = FP8 ? 32 : 64;
 constexpr float kLn2 = 0.6931471805599453f;
 // Of every 8 pairs of exponentials, this many are computed by the FMA-pipe
 // polynomial instead of the MUFU ex2 unit (balances the two pipes).
@@ -141,7 +148,7 @@ struct Params {
   int group;        // Hq / Hkv
   int pair_heads;   // 1: the two tiles are heads 2p, 2p+1 of one group
   int n_pairs;      // units per row group
-  int n_mgroups;    // row groups
+  int mg_hi;        // this launch covers row groups [mg_hi - n_units / n_pairs, mg_hi)
   int n_units;
   int causal, window;
   float scale_log2;  // logit scale * log2(e) (fp8: times both descales)
@@ -200,7 +207,7 @@ template <bool PAGED>
 __device__ __forceinline__ Unit get_unit(int u, const Params& p) {
   Unit w;
   int b_seq;
-  const int mg = p.n_mgroups - 1 - u / p.n_pairs;
+  const int mg = p.mg_hi - 1 - u / p.n_pairs;
   const int pr = u % p.n_pairs;
   if (p.pair_heads) {
     const int hp_per_b = p.Hq >> 1;
@@ -285,7 +292,7 @@ static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserv
 template <bool FP8, bool RSUM, bool FINE, bool E5M2 = false>
 __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
                                        uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
-                                       uint32_t (&pk_lo)[kBN / 4]) {
+                                       uint32_t (&pk_lo)[kBN / 2]) {
   const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
   float p0, p1;
   if ((q2 & 7) >= 8 - kEmuPairsPer8<FP8>) {
@@ -317,46 +324,58 @@ __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64
   } else {
     const uint32_t b = pack_bf16x2(p0, p1);
     pk[q2] = b;
-    if (RSUM) rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
+    float h0 = __uint_as_float(b << 16), h1 = __uint_as_float(b & 0xFFFF0000u);
+    if (FINE) {
+      const uint32_t bl = pack_bf16x2(p0 - h0, p1 - h1);  // P - h is exact in fp32
+      pk_lo[q2] = bl;
+      h0 += __uint_as_float(bl << 16);
+      h1 += __uint_as_float(bl & 0xFFFF0000u);
+    }
+    if (RSUM) rr2[q2 & 3] = add2(rr2[q2 & 3], f2(h0, h1));
   }
 }
 
 template <bool FP8, bool RSUM, bool FINE, int Q_LO, int Q_HI, bool E5M2 = false>
 __device__ __forceinline__ void p_pairs(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2, uint64_t (&rs2)[4],
-                                        uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2], uint32_t (&pk_lo)[kBN / 4]) {
+                                        uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2], uint32_t (&pk_lo)[kBN / 2]) {
 #pragma unroll
   for (int q2 = Q_LO; q2 < Q_HI; ++q2) p_pair<FP8, RSUM, FINE, E5M2>(q2, sr, sc2, nm2, rs2, rr2, pk, pk_lo);
 }
 
-// Fine e4m3 tiles: pairs [Q_LO, Q_HI) in chunks of 16 (32 keys), each chunk's
-// P and residual stored to TMEM at once (columns Q/2 on, at taddr and
-// taddr + kFineCol), so that the residual adds few live registers.
-template <bool RSUM, bool E5M2, int Q_LO, int Q_HI>
+// Fine tiles: pairs [Q_LO, Q_HI) in chunks of 8 TMEM columns (e4m3: 16 pairs,
+// bf16: 8), each chunk's P and residual stored to TMEM at once (at taddr and taddr + kFineCol; e4m3
+// packs two pairs per column, bf16 one), so that the residual adds few live
+// registers.
+template <bool FP8, bool RSUM, bool E5M2, int Q_LO, int Q_HI>
 __device__ __forceinline__ void p_pairs_fine(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
                                              uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
-                                             uint32_t (&pk_lo)[kBN / 4], uint32_t taddr) {
+                                             uint32_t (&pk_lo)[kBN / 2], uint32_t taddr) {
   if constexpr (Q_LO < Q_HI) {
-    constexpr int QE = Q_LO + 16 < Q_HI ? Q_LO + 16 : Q_HI;
-    p_pairs<true, RSUM, true, Q_LO, QE, E5M2>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
-    tmem_st_cols<Q_LO / 2, QE / 2>(taddr, pk);
-    tmem_st_cols<Q_LO / 2, QE / 2>(taddr + kFineCol, pk_lo);
-    p_pairs_fine<RSUM, E5M2, QE, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, taddr);
+    constexpr int CH = FP8 ? 16 : 8;  // pairs per chunk: 8 TMEM columns each way
+    constexpr int QE = Q_LO + CH < Q_HI ? Q_LO + CH : Q_HI;
+    constexpr int C0 = FP8 ? Q_LO / 2 : Q_LO, C1 = FP8 ? QE / 2 : QE;
+    p_pairs<FP8, RSUM, true, Q_LO, QE, E5M2>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+    tmem_st_cols<C0, C1>(taddr, pk);
+    tmem_st_cols<C0, C1>(taddr + kFineCol<FP8>, pk_lo);
+    p_pairs_fine<FP8, RSUM, E5M2, QE, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, taddr);
   }
 }
 
 // Is tile t of unit w a "fine" e4m3 tile (its first row sees < kFineKeys keys)?
-template <bool FP8, bool E5M2>
+// FINE: the kernel is built with the two-part product at all (without it,
+// the launch covers no tile that needs it; see run()).
+template <bool FP8, bool E5M2, bool FINE>
 __device__ __forceinline__ bool tile_fine(const Unit& w, int t, const Params& p) {
-  if (!FP8) return false;
-  if (E5M2) return true;  // 2 mantissa bits: every tile takes the residual product
+  if (!FINE) return false;
+  if (FP8 && E5M2) return true;  // 2 mantissa bits: every tile takes the residual product
   const int m0 = w.m0_of(t);
   if (m0 >= p.Lq) return false;
   int lo, hi;
   key_range(m0, w.lk, p, lo, hi);
-  return hi - lo < kFineKeys;
+  return hi - lo < (FP8 ? kFineKeys : kFineKeysBf16);
 }
 
-template <int D, bool FP8, bool PAGED, bool E5M2>
+template <int D, bool FP8, bool PAGED, bool E5M2, bool FINE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -593,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
         const Unit w = get_unit<PAGED>(u, p);
         if (w.nb <= 0) continue;
-        const bool fine0 = tile_fine<FP8, E5M2>(w, 0, p), fine1 = tile_fine<FP8, E5M2>(w, 1, p);
+        const bool fine0 = tile_fine<FP8, E5M2, FINE>(w, 0, p), fine1 = tile_fine<FP8, E5M2, FINE>(w, 1, p);
         ok = mbar_wait(&sm.q_full[0], nunit & 1, g) && mbar_wait(&sm.q_full[1], nunit & 1, g);
         if (!ok) break;
         // first K block
@@ -646,19 +665,25 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!ok) break;
             }
             tc_fence_after();
-            const bool fine = t ? fine1 : fine0;
+            // fine tiles: a second product with the residual of P (one loop
+            // body for both parts keeps the issuing thread's registers low)
+            const int parts = (t ? fine1 : fine0) ? 2 : 1;
             if (kSplitP) {
-              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, kSplitKeys / C::MMA_K, 0);
-              if (fine) issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, 0, kSplitKeys / C::MMA_K, kFineCol);
+#pragma unroll 1
+              for (int pt = 0; pt < parts; ++pt)
+                issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0 || pt > 0, 0, kSplitKeys / C::MMA_K,
+                         pt ? kFineCol<FP8> : 0u);
               ok = mbar_wait(&sm.p_full[t], pcnt & 1, g);
               if (!ok) break;
               tc_fence_after();
-              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS, 0);
-              if (fine)
-                issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS, kFineCol);
+#pragma unroll 1
+              for (int pt = 0; pt < parts; ++pt)
+                issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, kSplitKeys / C::MMA_K, C::PV_KSTEPS,
+                         pt ? kFineCol<FP8> : 0u);
             } else {
-              issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0, 0, C::PV_KSTEPS, 0);
-              if (fine) issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, true, 0, C::PV_KSTEPS, kFineCol);
+#pragma unroll 1
+              for (int pt = 0; pt < parts; ++pt)
+                issue_pv(t, kv_addr0 + sv * C::TILE_BYTES, j > 0 || pt > 0, 0, C::PV_KSTEPS, pt ? kFineCol<FP8> : 0u);
             }
             if (!has_next) tc_commit(&sm.o_full[t]);
             if (has_next) {
@@ -708,9 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the MMA multiplies (normalises O so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
       // fine e4m3 tile: exact running max, P scaled by 2^kFineShift, residual product
-      const bool fine = tile_fine<FP8, E5M2>(w, t, p);
-      const float thr = fine ? 0.f : kRescaleThreshold;
-      const float shift = fine ? kFineShift : 0.f;
+      const bool fine = tile_fine<FP8, E5M2, FINE>(w, t, p);
+      // (8-bit P only: exact running max and P scaled by 2^kFineShift)
+      const float thr = (FP8 && fine) ? 0.f : kRescaleThreshold;
+      const float shift = (FP8 && fine) ? kFineShift : 0.f;
       if (w.nb > 0) {
         int lo, hi;
         key_range(row, w.lk, p, lo, hi);
@@ -753,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // four independent packed accumulators each.
           uint64_t rs2[4] = {0, 0, 0, 0}, rr2[4] = {0, 0, 0, 0};
           uint32_t pk[kBN / 2];     // P of the block, packed for the MMA
-          uint32_t pk_lo[kBN / 4];  // fine e4m3 tiles: the rounding residual of P
+          uint32_t pk_lo[kBN / 2];  // fine tiles: the rounding residual of P
           // Rescale the accumulator when the running max moved.  The previous
           // P.V of this tile has completed: it was issued before this S.
           auto rescale_o = [&]() {
@@ -770,12 +796,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           };
           // P of pairs [Q_LO, Q_HI) into TMEM: bf16 one key pair per column,
-          // e4m3 two pairs (and in fine tiles the residual kFineCol columns on).
+          // e4m3 two pairs (and in fine tiles the residual kFineCol columns
+          // on; e5m2 tiles are always fine).
           auto p_part = [&](auto q_lo_c, auto q_hi_c) {
             constexpr int Q_LO = decltype(q_lo_c)::value, Q_HI = decltype(q_hi_c)::value;
             constexpr int C0 = FP8 ? Q_LO / 2 : Q_LO, C1 = FP8 ? Q_HI / 2 : Q_HI;
-            if (FP8 && (E5M2 || fine)) {
-              p_pairs_fine<kRsum, E5M2, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
+            if (fine) {
+              p_pairs_fine<FP8, kRsum, E5M2, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
             } else {
               p_pairs<FP8, kRsum, false, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
               tmem_st_cols<C0, C1>(tS, pk);
@@ -871,19 +898,39 @@ bool encode_pool(CUtensorMap* map, const void* pool, bool fp8, int D, int num_pa
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, bool PAGED, bool E5M2 = false>
-int run(const PrefillArgs& a, cudaStream_t stream) {
+// Visible-key count of query row i on the host, as key_range().
+int host_key_count(int i, int lk, const PrefillArgs& a) {
+  if (!a.causal) return lk;
+  int h = i + (lk - a.Lq) + 1;
+  h = h < 0 ? 0 : (h > lk ? lk : h);
+  const int lo = (a.window > 0 && h - a.window > 0) ? h - a.window : 0;
+  return h - lo;
+}
+
+template <int D, bool FP8, bool PAGED, bool E5M2, bool FINE>
+int launch_range(const PrefillArgs& a, Params p, int mg_lo, int mg_hi, const CUtensorMap& tq,
+                 const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
   using C = Cfg<D, FP8, E5M2>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
   if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(prefill_kernel<D, FP8, PAGED, E5M2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::SMEM_BYTES);
+    err = cudaFuncSetAttribute(prefill_kernel<D, FP8, PAGED, E5M2, FINE>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return fail_cuda("prefill: cudaFuncSetAttribute", err);
     attr_set[dev] = true;
   }
+  p.mg_hi = mg_hi;
+  p.n_units = p.n_pairs * (mg_hi - mg_lo);
+  const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+  prefill_kernel<D, FP8, PAGED, E5M2, FINE><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  err = cudaGetLastError();
+  return err == cudaSuccess ? 0 : fail_cuda("prefill: launch", err);
+}
+
+template <int D, bool FP8, bool PAGED, bool E5M2 = false>
+int run(const PrefillArgs& a, cudaStream_t stream) {
   Params p{};
   p.o = a.o;
   p.lse = a.lse;
@@ -894,14 +941,14 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   p.Lk = a.Lk;
   p.group = a.Hq / a.Hkv;
   p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
+  int n_mgroups;
   if (p.pair_heads) {
     p.n_pairs = a.B * (a.Hq / 2);
-    p.n_mgroups = (a.Lq + kBM - 1) / kBM;
+    n_mgroups = (a.Lq + kBM - 1) / kBM;
   } else {
     p.n_pairs = a.B * a.Hq;
-    p.n_mgroups = (a.Lq + 2 * kBM - 1) / (2 * kBM);
+    n_mgroups = (a.Lq + 2 * kBM - 1) / (2 * kBM);
   }
-  p.n_units = p.n_pairs * p.n_mgroups;
   p.causal = a.causal;
   p.window = a.window > 0 ? a.window : 0;
   const float log2e = 1.4426950408889634f;
@@ -918,27 +965,51 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
   p.num_pages = a.num_pages;
 
   CUtensorMap tq, tk, tv;
-  if (PAGED) {
+  if constexpr (PAGED) {
     if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq))
       return fail_cuda("prefill: tensor map (q)", cudaErrorInvalidValue);
     if (!encode_pool(&tk, a.k, FP8, D, a.num_pages, a.Hkv) || !encode_pool(&tv, a.v, FP8, D, a.num_pages, a.Hkv))
       return fail_cuda("prefill: tensor map (pool)", cudaErrorInvalidValue);
-    const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
-    prefill_kernel<D, FP8, PAGED, E5M2><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-    err = cudaGetLastError();
-    return err == cudaSuccess ? 0 : fail_cuda("prefill (paged): launch", err);
+    // Sequence lengths are device data: one launch that decides per tile.
+    return launch_range<D, FP8, PAGED, E5M2, true>(a, p, 0, n_mgroups, tq, tk, tv, stream);
+  } else {
+    const bool have_k = a.Lk > 0;
+    if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq))
+      return fail_cuda("prefill: tensor map (q)", cudaErrorInvalidValue);
+    // With no keys nothing is loaded from K/V; describe Q instead of an empty tensor.
+    const void* kb = have_k ? a.k : a.q;
+    const void* vb = have_k ? a.v : a.q;
+    const int rows = have_k ? a.Lk : a.Lq;
+    const uint64_t outer = have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq;
+    if (!encode_3d(&tk, kb, FP8, D, rows, outer)) return fail_cuda("prefill: tensor map (k)", cudaErrorInvalidValue);
+    if (!encode_3d(&tv, vb, FP8, D, rows, outer)) return fail_cuda("prefill: tensor map (v)", cudaErrorInvalidValue);
+    if constexpr (FP8 && E5M2) {
+      return launch_range<D, FP8, PAGED, E5M2, true>(a, p, 0, n_mgroups, tq, tk, tv, stream);
+    } else {
+      // Tiles that take the two-part product ("fine": the first row sees
+      // fewer keys than the threshold) are the leading row groups: a row's key
+      // count never decreases along the rows.  They run in a kernel built with
+      // that product; the rest in one built without it, whose softmax and MMA
+      // issue then carry none of its code (that code alone measured ~6 % on
+      // the GQA causal workload).
+      const int thr = FP8 ? kFineKeys : kFineKeysBf16;
+      int mg_fine = 0;
+      while (mg_fine < n_mgroups) {
+        bool any = false;
+        for (int t = 0; t < 2; ++t) {
+          const int m0 = p.pair_heads ? mg_fine * kBM : (2 * mg_fine + t) * kBM;
+          if (m0 < a.Lq && host_key_count(m0, a.Lk, a) < thr) any = true;
+        }
+        if (!any) break;
+        ++mg_fine;
+      }
+      int st = 0;
+      if (mg_fine > 0) st = launch_range<D, FP8, PAGED, E5M2, true>(a, p, 0, mg_fine, tq, tk, tv, stream);
+      if (st == 0 && mg_fine < n_mgroups)
+        st = launch_range<D, FP8, PAGED, E5M2, false>(a, p, mg_fine, n_mgroups, tq, tk, tv, stream);
+      return st;
+    }
   }
-  const bool have_k = a.Lk > 0;
-  if (!encode_3d(&tq, a.q, FP8, D, a.Lq, (uint64_t)a.B * a.Hq)) return fail_cuda("prefill: tensor map (q)", cudaErrorInvalidValue);
-  // With no keys nothing is loaded from K/V; describe Q instead of an empty tensor.
-  if (!encode_3d(&tk, have_k ? a.k : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
-    return fail_cuda("prefill: tensor map (k)", cudaErrorInvalidValue);
-  if (!encode_3d(&tv, have_k ? a.v : a.q, FP8, D, have_k ? a.Lk : a.Lq, have_k ? (uint64_t)a.B * a.Hkv : (uint64_t)a.B * a.Hq))
-    return fail_cuda("prefill: tensor map (v)", cudaErrorInvalidValue);
-  const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
-  prefill_kernel<D, FP8, PAGED, E5M2><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-  err = cudaGetLastError();
-  return err == cudaSuccess ? 0 : fail_cuda("prefill: launch", err);
 }
 
 }  // namespace

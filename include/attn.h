@@ -4,7 +4,7 @@
  *
  * Operations, all on one GPU:
  *
- *   attn_fwd / attn_fwd_fp8 / attn_fwd_e5m2
+ *   attn_fwd / attn_fwd_fp8 / attn_fwd_e5m2 / attn_fwd_mla
  *                             fused, tiled scaled-dot-product attention
  *                             O = softmax(scale * Q K^T + mask) V, with the
  *                             per-row log-sum-exp, computed with the online
@@ -36,6 +36,8 @@
  *     kernel).
  *   - "注意力机制深度优化" (kler.cn) §一.1 (FP8 e4m3), §一.2 (skipping the
  *     upper-right causal triangle), §四.2 (FP8 e5m2).
+ *   - "高效多头潜在注意力解码技术：Flash MLA深度解析" (developer.baidu.com)
+ *     §2.1: queries and keys in a latent dimension, values in their own.
  *
  * Conventions shared by every entry point
  *   - Pointers are DEVICE pointers unless stated otherwise.  The caller owns
@@ -156,6 +158,29 @@ ATTN_API int attn_fwd_e5m2(const void* q, const void* k, const void* v, void* o,
                            float scale, int causal, int window,
                            float q_descale, float k_descale, float v_descale,
                            attn_stream_t stream);
+
+/*
+ * attn_fwd_mla -- bf16 attention forward whose queries and keys have another
+ * width than the values, up to 256: attention in a latent space, where q and
+ * k are projections to a latent dimension (64-256 on the page) and v to its
+ * own value dimension (latent projection of the page "高效多头潜在注意力解码
+ * 技术：Flash MLA深度解析", §2.1).
+ *
+ *   q    [B, Hq,  Lq, D_qk] bf16     k [B, Hkv, Lk, D_qk] bf16
+ *   v    [B, Hkv, Lk, D_v]  bf16
+ *   o    [B, Hq,  Lq, D_v]  bf16 (written)
+ *   lse  [B, Hq,  Lq]       fp32 (written; may be NULL)
+ *
+ * Masks, GQA/MQA head mapping, scale, precision and empty-row behaviour as
+ * attn_fwd.  One 128-row query tile per SM with 64-key K/V blocks (two
+ * 128-row accumulators of 256 columns do not fit the tensor memory), so for
+ * D_qk = D_v in {64, 128} attn_fwd is the faster call.
+ * Supported: D_qk, D_v in {64, 128, 192, 256} (ATTN_ERR_UNSUPPORTED
+ * otherwise); other checks as attn_fwd.
+ */
+ATTN_API int attn_fwd_mla(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int Lq, int Lk, int D_qk, int D_v,
+                          float scale, int causal, int window, attn_stream_t stream);
 
 /*
  * attn_bwd_workspace_bytes -- scratch attn_bwd needs: an fp32 dQ accumulator

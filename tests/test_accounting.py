@@ -63,3 +63,16 @@ def test_decode_accounting():
 
 def test_prefill_shape_fields():
     assert isinstance(GQA_CAUSAL, PrefillShape) and GQA_CAUSAL.Hq // GQA_CAUSAL.Hkv == 4
+
+
+def test_latent_shapes_count_both_widths():
+    """D_qk != D_v: Q.K^T costs 2*D_qk per visible pair and P.V 2*D_v; K is
+    read at width D_qk, V at D_v, O written at D_v."""
+    from workloads import LATENT_192_128
+    s = LATENT_192_128
+    pairs = 4096 * 4097 // 2
+    assert prefill_flops(s) == 2 * (192 + 128) * 4 * 32 * pairs
+    q = 4 * 32 * 4096 * 192 * 2
+    kv = 4 * 8 * 4096 * (192 + 128) * 2
+    o = 4 * 32 * 4096 * 128 * 2
+    assert prefill_bytes(s) == q + kv + o + 4 * 32 * 4096 * 4

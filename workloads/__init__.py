@@ -8,7 +8,8 @@ bit-identical inputs.
 Recipe (one ``torch.Generator`` per call, seeded by the caller):
 
 * prefill: q, k, v drawn in that order, fp32 N(0, 1), cast round-to-nearest-even
-  to bf16, contiguous ``[B, H, L, D]`` (the ``(batch, num_heads, seqlen,
+  to bf16, contiguous ``[B, H, L, D]`` (v ``[B, H, L, Dv]`` where the value
+  width differs) (the ``(batch, num_heads, seqlen,
   head_dim)`` layout of the HF-Llama ``view(...).transpose(1, 2)`` code on the
   zeeklog page "LLM 中的 Attention 实现及优化", GQA section).
 * FP8 prefill: the same fp32 draws, each tensor quantised to ``float8_e4m3fn``
@@ -49,10 +50,15 @@ class PrefillShape:
     causal: bool
     window: int = 0          # 0 = no window
     fp8: bool = False
+    Dv: int = 0              # value width; 0 = D (queries and keys have width D)
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.D)
+
+    @property
+    def dv(self) -> int:
+        return self.Dv or self.D
 
 
 @dataclasses.dataclass(frozen=True)
@@ -81,6 +87,14 @@ FP8_CAUSAL = PrefillShape("fp8_causal_B1_H32_L32768_D128", B=1, Hq=32, Hkv=32, L
 
 WORKLOADS = [TINY_MHA, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, FP8_CAUSAL]
 
+# Latent-space shapes (queries and keys of width 64-256, values of their own
+# width: the latent projection of the Flash MLA page, §2.1), measured beside
+# the five workloads above with the seeds of workloads 1 and 3.
+LATENT_192_128 = PrefillShape("latent_causal_B4_H32_G4_L4096_Dqk192_Dv128", B=4, Hq=32, Hkv=8, Lq=4096, Lk=4096,
+                              D=192, causal=True, Dv=128)
+LATENT_256 = PrefillShape("latent_causal_B4_H32_G4_L4096_D256", B=4, Hq=32, Hkv=8, Lq=4096, Lk=4096, D=256,
+                          causal=True)
+
 
 def seed_of(index: int) -> int:
     return 1000 + index
@@ -101,7 +115,7 @@ def prefill_inputs(shape: PrefillShape, seed: int):
     g = _gen(seed)
     q = _normal(g, (shape.B, shape.Hq, shape.Lq, shape.D)).to(torch.bfloat16)
     k = _normal(g, (shape.B, shape.Hkv, shape.Lk, shape.D)).to(torch.bfloat16)
-    v = _normal(g, (shape.B, shape.Hkv, shape.Lk, shape.D)).to(torch.bfloat16)
+    v = _normal(g, (shape.B, shape.Hkv, shape.Lk, shape.dv)).to(torch.bfloat16)
     return q, k, v
 
 

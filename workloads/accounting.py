@@ -9,9 +9,10 @@ from . import DecodeShape, PrefillShape
 
 
 def prefill_flops(shape: PrefillShape) -> float:
-    """FLOPs as actually required: 4*D per visible (query, key) pair per head
-    (2*D for Q.K^T, 2*D for P.V)."""
-    return 4.0 * shape.D * shape.B * shape.Hq * visible_pairs(shape.Lq, shape.Lk, shape.causal, shape.window)
+    """FLOPs as actually required: 2*D + 2*Dv per visible (query, key) pair
+    per head (2*D for Q.K^T, 2*Dv for P.V; 4*D when the widths agree)."""
+    return 2.0 * (shape.D + shape.dv) * shape.B * shape.Hq * visible_pairs(shape.Lq, shape.Lk, shape.causal,
+                                                                          shape.window)
 
 
 def visible_pairs(Lq: int, Lk: int, causal: bool, window: int) -> int:
@@ -33,8 +34,8 @@ def prefill_bytes(shape: PrefillShape) -> float:
     """Algorithmic HBM bytes: read Q, K, V once, write O and LSE once."""
     el = 1 if shape.fp8 else 2
     q = shape.B * shape.Hq * shape.Lq * shape.D * el
-    kv = 2 * shape.B * shape.Hkv * shape.Lk * shape.D * el
-    o = shape.B * shape.Hq * shape.Lq * shape.D * 2
+    kv = shape.B * shape.Hkv * shape.Lk * (shape.D + shape.dv) * el
+    o = shape.B * shape.Hq * shape.Lq * shape.dv * 2
     lse = shape.B * shape.Hq * shape.Lq * 4
     return float(q + kv + o + lse)
 
