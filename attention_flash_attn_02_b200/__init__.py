@@ -70,6 +70,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.attn_decode_paged.restype = c_int
     lib.attn_decode_paged_multi.argtypes = [c_void_p] * 7 + [c_int] * 8 + [c_float, c_void_p, c_size_t, c_void_p]
     lib.attn_decode_paged_multi.restype = c_int
+    lib.attn_decode_paged_mla.argtypes = [c_void_p] * 7 + [c_int] * 9 + [c_float, c_void_p, c_size_t, c_void_p]
+    lib.attn_decode_paged_mla.restype = c_int
     lib.attn_prefill_paged.argtypes = [c_void_p] * 7 + [c_int] * 8 + [c_float, c_int, c_void_p]
     lib.attn_prefill_paged.restype = c_int
     lib.attn_kv_append.argtypes = [c_void_p] * 6 + [c_int] * 7 + [c_void_p]
@@ -267,6 +269,40 @@ def attn_decode_paged_multi(q, k_pages, v_pages, block_table, seq_lens, scale: O
                                      float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _stream_handle(stream))
     _check(st, "attn_decode_paged_multi")
+    return o, lse
+
+
+def attn_decode_paged_mla(q, k_pages, v_pages, block_table, seq_lens, scale: Optional[float] = None,
+                          o=None, lse=None, workspace=None, stream=None):
+    """Paged decode with query/key width D_qk and value width D_v (each 64,
+    128, 192 or 256).  q [B,Hq,q_len,D_qk] bf16 (the last q_len cached tokens);
+    k_pages [P,16,Hkv,D_qk], v_pages [P,16,Hkv,D_v] bf16; block_table
+    [B,max_pages] int32; seq_lens [B] int32.  The default scale is
+    1/sqrt(D_qk).  Returns (o bf16 [B,Hq,q_len,D_v], lse fp32 [B,Hq,q_len])."""
+    import torch
+    lib = load()
+    B, Hq, q_len, Dqk = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    Dv = v_pages.shape[3]
+    max_pages = block_table.shape[1]
+    if k_pages.shape[3] != Dqk or v_pages.shape[:3] != k_pages.shape[:3]:
+        raise ValueError("attn_decode_paged_mla: k_pages must be [P,16,Hkv,D_qk] and v_pages [P,16,Hkv,D_v]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dqk)
+    if o is None:
+        o = torch.empty((B, Hq, q_len, Dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, q_len), dtype=torch.float32, device=q.device)
+    need = lib.attn_decode_workspace_bytes(B, Hq * q_len, max(max_pages, 1), Dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("attn_decode_paged_mla: block_table and seq_lens must be int32")
+    st = lib.attn_decode_paged_mla(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                                   _ptr(o), _ptr(lse), B, Hq, Hkv, q_len, Dqk, Dv, page_size, num_pages, max_pages,
+                                   float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream_handle(stream))
+    _check(st, "attn_decode_paged_mla")
     return o, lse
 
 

@@ -151,9 +151,9 @@ namespace attn {
 // (B == 0 included: nothing to launch), else the status to return.
 int validate_decode(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
                     const int* seq_lens, const void* o, const float* lse, int B, int Hq, int Hkv, int q_len, int D,
-                    int page_size, int num_pages, int max_pages_per_seq, float scale) {
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages_per_seq < 0 ||
-      q_len <= 0)
+                    int Dv, int page_size, int num_pages, int max_pages_per_seq, float scale) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Dv <= 0 || page_size <= 0 || num_pages < 0 ||
+      max_pages_per_seq < 0 || q_len <= 0)
     return ATTN_ERR_INVALID;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
   if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;
@@ -164,24 +164,25 @@ int validate_decode(const void* q, const void* k_pages, const void* v_pages, con
     return ATTN_ERR_INVALID;
   if (num_pages > 0 && (!k_pages || !v_pages || !aligned16(k_pages) || !aligned16(v_pages)))
     return ATTN_ERR_INVALID;
-  if (D != 128 || page_size != 16 || (Hq / Hkv) * q_len > 128) return ATTN_ERR_UNSUPPORTED;
+  auto ok_dim = [](int d) { return d == 64 || d == 128 || d == 192 || d == 256; };
+  if (!ok_dim(D) || !ok_dim(Dv) || page_size != 16 || (Hq / Hkv) * q_len > 128) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 }  // namespace attn
 
 namespace {
 int decode_checked(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
-                   const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int q_len, int D,
+                   const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int q_len, int D, int Dv,
                    int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
                    size_t workspace_bytes, attn_stream_t stream) {
-  const int st = validate_decode(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D,
+  const int st = validate_decode(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D, Dv,
                                  page_size, num_pages, max_pages_per_seq, scale);
   if (st != ATTN_OK || B == 0) return st;
   const int mp = max_pages_per_seq > 0 ? max_pages_per_seq : 1;
-  const size_t need = attn_decode_workspace_bytes(B, Hq * q_len, mp, D);
+  const size_t need = attn_decode_workspace_bytes(B, Hq * q_len, mp, Dv);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_INVALID;
   DecodeArgs a{q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size, num_pages,
-               max_pages_per_seq, scale, workspace, workspace_bytes, q_len};
+               max_pages_per_seq, scale, workspace, workspace_bytes, q_len, Dv};
   return launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
@@ -190,7 +191,7 @@ ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v
                                const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
                                int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
                                size_t workspace_bytes, attn_stream_t stream) {
-  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, 1, D, page_size,
+  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, 1, D, D, page_size,
                         num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
 }
 
@@ -199,7 +200,15 @@ ATTN_API int attn_decode_paged_multi(const void* q, const void* k_pages, const v
                                      int Hq, int Hkv, int q_len, int D, int page_size, int num_pages,
                                      int max_pages_per_seq, float scale, void* workspace, size_t workspace_bytes,
                                      attn_stream_t stream) {
-  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D, page_size,
+  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D, D, page_size,
+                        num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
+}
+
+ATTN_API int attn_decode_paged_mla(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                                   const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int q_len,
+                                   int D_qk, int D_v, int page_size, int num_pages, int max_pages_per_seq,
+                                   float scale, void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+  return decode_checked(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, q_len, D_qk, D_v, page_size,
                         num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
 }
 

@@ -81,7 +81,7 @@ ATTN_API int attn_decode_paged_noalloc(const void* q, const void* k_pages, const
                                        float scale, attn_stream_t stream) {
   // The same argument checks as attn_decode_paged, in the same order, so the
   // two return the same status for the same arguments.
-  int st = validate_decode(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, 1, D, page_size,
+  int st = validate_decode(q, k_pages, v_pages, block_table, seq_lens, o, lse, B, Hq, Hkv, 1, D, D, page_size,
                            num_pages, max_pages_per_seq, scale);
   if (st != ATTN_OK) return st;
   // Set-up (first call per device, B == 0 included): the array's address.

@@ -42,37 +42,58 @@
 namespace attn {
 namespace {
 
-constexpr int kD = 128;
 constexpr int kPage = 16;
-// Blocks of 4 pages (64 tokens) in a 3-stage ring of 96 KB, two CTAs per SM
-// with 256 TMEM columns each.  (Measured on B200 against 2-page blocks with
-// two CTAs per SM and 8-page blocks with one: 4 pages was fastest.)
+// Blocks of 4 pages (64 tokens) in a ring of up to 3 stages.  (Measured on
+// B200 at D = 128 against 2-page blocks with two CTAs per SM and 8-page blocks
+// with one: 4 pages was fastest.)  Features go in boxes of 64 (128 bytes,
+// one row of the 128-byte swizzle): D_qk / 64 boxes of K and D_v / 64 of V.
 constexpr int kBlkPages = 4;                    // pages per block
 constexpr int kBlkTok = kBlkPages * kPage;      // 64 tokens per block
-constexpr int kHalf = kBlkTok * 128;            // a block's 64-feature half (bf16): 8 KB
-constexpr int kPageHalf = kPage * 128;          // one page's 64-feature half: 2 KB
-constexpr int kStageBytes = 4 * kHalf;          // K half 0, K half 1, V half 0, V half 1
-constexpr int kCtasPerSm = 2;
+constexpr int kBox = kBlkTok * 128;             // a block's 64-feature box (bf16): 8 KB
+constexpr int kPageBox = kPage * 128;           // one page's 64-feature box: 2 KB
 constexpr int kMaxStages = 3;                   // ring stages (fewer when the query tile is large)
 constexpr int kThreads = 192;                   // warps 0-3 softmax, 4 producer, 5 MMA
 constexpr int kMaxGroup = 128;                  // query rows per K/V head tile: group * q_len
-constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmS0 = 0, kTmS1 = kBlkTok, kTmO = 2 * kBlkTok;
-static_assert(kTmO + kD <= kTmemCols, "TMEM budget");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr uint32_t kIdescPV = make_idesc(1u, 128, kD, true);
+constexpr int kSmemPerSm = 233472;  // shared memory of an SM, 1 KB of it reserved per CTA
+// Segments of sequences whose first query token sees fewer than kFineKeys
+// cached tokens multiply V by P in two bf16 parts, P rounded and its rounding
+// residual (TMEM columns 32-63 of the S buffer; P of a 64-token block fills
+// 0-31): on a row of a few keys, rounding P to bf16 alone moves O by up to
+// ~2^-9 of the spread of its V values, which with the bf16 rounding of O can
+// pass 1e-2.  Decided from the sequence's page count P, which every role
+// already has (its capacity P * 16 bounds the length): P * 16 - q_len + 1 <
+// kFineKeys.
+constexpr int kFineKeys = 256;
+constexpr uint32_t kFineCol = 32;
+__device__ __forceinline__ bool seg_fine(int pages, int q_len) { return pages * kPage - q_len + 1 < kFineKeys; }
+
+// Per-width constants: query/key width DQK, value width DV (64..256).
+template <int DQK, int DV>
+struct DecCfg {
+  static constexpr int KB = DQK / 64, VB = DV / 64;         // feature boxes of K and V
+  static constexpr int STAGE = (KB + VB) * kBox;            // K boxes, then V boxes
+  // TMEM: two S buffers of 64 columns and O of DV columns; 256 columns let
+  // two CTAs share an SM, wider O takes all 512 (one CTA per SM).
+  static constexpr uint32_t TMEM_COLS = kTmO + DV <= 256 ? 256u : 512u;
+  static constexpr int TMEM_CTAS = 512 / (int)TMEM_COLS;    // CTAs an SM's TMEM holds
+  static constexpr uint32_t IDESC_PV = make_idesc(1u, 128, DV, true);
+  static_assert(DQK % 64 == 0 && DV % 64 == 0 && DQK <= 256 && DV <= 256, "widths 64..256 in steps of 64");
+  static_assert(kTmO + DV <= TMEM_COLS, "TMEM budget");
+};
 
 struct SplitParams {
   const int* block_table;
   const int* seq_lens;
-  float* ws_o;    // [B * Hq][S][kD] normalised partial outputs
+  float* ws_o;    // [B * Hq][S][D_v] normalised partial outputs
   float* ws_lse;  // [B * Hq][S] log2-sum-exp of each partial
   int B, Hq, Hkv, group, num_pages, max_pages, max_segs;
   int q_len;       // query tokens per sequence: the last q_len cached ones
   int rows;        // query rows per (sequence, K/V head): group * q_len
-  int q_half;      // bytes of one 64-feature half of a query tile
+  int q_box;       // bytes of one 64-feature box of a query tile
   int q_slots;     // query tiles in flight (1 or 2)
   int stages;      // K/V ring stages (2 or 3)
   int sm_warps;    // softmax warps with rows: ceil(rows / 32)
@@ -94,20 +115,21 @@ struct DecSmem {
 constexpr int kBarBytes = 256;
 static_assert(sizeof(DecSmem) <= kBarBytes, "barrier block exceeds its reserve");
 // Shared memory: [query slot 0][query slot 1][ring][barriers], the base
-// 1024-byte aligned.  Two CTAs must fit on an SM (233472 bytes, 1 KB of it
-// reserved per CTA) and a third must not (TMEM holds two CTAs' columns).
-// Query slots (one or two, each two 64-feature halves) and ring stages are
-// chosen per call so that two CTAs fit on an SM: the deepest ring first, then
-// the second query slot (it only hides the query load at a segment switch).
-__host__ __device__ constexpr int dec_smem_bytes(int q_half, int q_slots, int stages) {
-  return q_slots * 2 * q_half + stages * kStageBytes + kBarBytes;
+// 1024-byte aligned.  Query slots (one or two, each DQK / 64 boxes) and ring
+// stages are chosen per call (host side) so that as many CTAs share an SM as
+// its TMEM holds (two at D_v <= 128): the deepest ring first, then the second
+// query slot (it only hides the query load at a segment switch); where even
+// the smallest layout does not fit twice, one CTA per SM.  A launch never
+// asks for so little shared memory that more CTAs than the TMEM holds could
+// share an SM (their allocation would wait).
+template <int DQK, int DV>
+__host__ __device__ constexpr int dec_smem_bytes(int q_box, int q_slots, int stages) {
+  return q_slots * DecCfg<DQK, DV>::KB * q_box + stages * DecCfg<DQK, DV>::STAGE + kBarBytes;
 }
-constexpr bool two_fit(int bytes) { return kCtasPerSm * (bytes + 1024) <= 233472; }
-static_assert(two_fit(dec_smem_bytes(32 * 128, 2, kMaxStages)), "the MQA tile keeps the full layout");
-static_assert(two_fit(dec_smem_bytes(kMaxGroup * 128, 1, 2)), "the largest tile still fits twice per SM");
-// TMEM holds two CTAs' columns: a launch never asks for so little shared
-// memory that a third CTA would fit on an SM (its allocation would wait).
-constexpr int kMinSmem = 233472 / (kCtasPerSm + 1) - 1024 + 16;
+constexpr bool fits(int bytes, int ctas) { return ctas * (bytes + 1024) <= kSmemPerSm; }
+static_assert(fits(dec_smem_bytes<128, 128>(32 * 128, 2, kMaxStages), 2), "the MQA tile keeps the full layout");
+static_assert(fits(dec_smem_bytes<128, 128>(kMaxGroup * 128, 1, 2), 2), "the largest tile still fits twice per SM");
+static_assert(fits(dec_smem_bytes<256, 256>(kMaxGroup * 128, 1, 2), 1), "the widest tile fits once per SM");
 
 // K/V pages are read once per call, so their TMA loads carry an L2
 // evict-first policy: they then do not push out the small data that is read
@@ -219,6 +241,42 @@ struct CombineParams {
 // (the same partition the split kernel used); after the wait, lane s reads
 // segment s's log2-sum-exp while every lane reads its 4 features of up to 8
 // partials at once.
+// F consecutive fp32 features from global memory (L2, bypassing L1), in
+// 16-byte loads where F allows, else 8-byte ones.
+template <int F>
+__device__ __forceinline__ void ld_feats(const float* src, float (&v)[F]) {
+  if constexpr (F % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < F / 4; ++i) {
+      const float4 t = __ldcg(reinterpret_cast<const float4*>(src) + i);
+      v[4 * i] = t.x;
+      v[4 * i + 1] = t.y;
+      v[4 * i + 2] = t.z;
+      v[4 * i + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < F / 2; ++i) {
+      const float2 t = __ldcg(reinterpret_cast<const float2*>(src) + i);
+      v[2 * i] = t.x;
+      v[2 * i + 1] = t.y;
+    }
+  }
+}
+// F bf16 features (F / 2 packed pairs) to global memory.
+template <int F>
+__device__ __forceinline__ void st_feats(__nv_bfloat16* dst, const uint32_t (&pk)[F / 2]) {
+  if constexpr (F == 8) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  } else if constexpr (F == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < F / 2; ++i) reinterpret_cast<uint32_t*>(dst)[i] = pk[i];
+  }
+}
+
+template <int DV>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
   // The next decode's split kernel (a programmatic dependent) may launch and
   // set up while this grid runs; it waits for this grid before reading or
@@ -256,28 +314,34 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the split kernel's partials are complete
-  const float* base_o = p.ws_o + (size_t)gw * p.max_segs * kD + lane * 4;
+  constexpr int F = DV / 32;  // features per lane
+  const float* base_o = p.ws_o + (size_t)gw * p.max_segs * DV + lane * F;
   const float* base_l = p.ws_lse + (size_t)gw * p.max_segs;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float acc[F];
+#pragma unroll
+  for (int f = 0; f < F; ++f) acc[f] = 0.f;
   float M = -INFINITY, L = 0.f;
   for (int s0 = 0; s0 < nseg; s0 += 32) {
     const int n = nseg - s0 < 32 ? nseg - s0 : 32;
     const float l2 = lane < n ? __ldcg(base_l + s0 + lane) : -INFINITY;
-    float4 v[8];
+    float v[8][F];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      v[u] = u < n ? __ldcg(reinterpret_cast<const float4*>(base_o + (size_t)(s0 + u) * kD))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < 8; ++u) {
+      if (u < n) {
+        ld_feats<F>(base_o + (size_t)(s0 + u) * DV, v[u]);
+      } else {
+#pragma unroll
+        for (int f = 0; f < F; ++f) v[u][f] = 0.f;
+      }
+    }
     float gm = l2;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
     const float Mn = fmaxf(M, gm);
     if (Mn == -INFINITY) continue;
     const float scale_old = (M == -INFINITY) ? 0.f : ex2_approx(M - Mn);
-    acc.x *= scale_old;
-    acc.y *= scale_old;
-    acc.z *= scale_old;
-    acc.w *= scale_old;
+#pragma unroll
+    for (int f = 0; f < F; ++f) acc[f] *= scale_old;
     L *= scale_old;
     M = Mn;
     const float w = (l2 == -INFINITY) ? 0.f : ex2_approx(l2 - M);
@@ -289,50 +353,50 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     for (int u = 0; u < 8; ++u) {
       const float wv = __shfl_sync(0xffffffffu, w, u);
       if (u < n) {
-        acc.x += wv * v[u].x;
-        acc.y += wv * v[u].y;
-        acc.z += wv * v[u].z;
-        acc.w += wv * v[u].w;
+#pragma unroll
+        for (int f = 0; f < F; ++f) acc[f] += wv * v[u][f];
       }
     }
     for (int u = 8; u < n; ++u) {  // more than 8 segments in this group of 32
-      const float4 vv = __ldcg(reinterpret_cast<const float4*>(base_o + (size_t)(s0 + u) * kD));
+      float vv[F];
+      ld_feats<F>(base_o + (size_t)(s0 + u) * DV, vv);
       const float wv = __shfl_sync(0xffffffffu, w, u);
-      acc.x += wv * vv.x;
-      acc.y += wv * vv.y;
-      acc.z += wv * vv.z;
-      acc.w += wv * vv.w;
+#pragma unroll
+      for (int f = 0; f < F; ++f) acc[f] += wv * vv[f];
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  uint2 packed;
-  packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-  packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-  *reinterpret_cast<uint2*>(p.o + (size_t)gw * kD + lane * 4) = packed;
+  uint32_t pk[F / 2];
+#pragma unroll
+  for (int f = 0; f < F / 2; ++f) pk[f] = pack_bf16x2(acc[2 * f] * inv, acc[2 * f + 1] * inv);
+  st_feats<F>(p.o + (size_t)gw * DV + lane * F, pk);
   if (lane == 0 && p.lse) p.lse[gw] = (L > 0.f) ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+template <int DQK, int DV>
+__global__ void __launch_bounds__(kThreads, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
+  using C = DecCfg<DQK, DV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t base = smem_u32(smem_raw);
   // This grid is launched as a programmatic dependent of the kernel before it
-  // in the stream, so that its launch and the set-up below (barriers, TMEM)
-  // overlap that kernel's tail.  That kernel may write any of the inputs or
-  // read the workspace, so nothing global is touched before
-  // griddepcontrol.wait.
+  // in the stream, so that its launch, the set-up below (barriers, TMEM) and
+  // the work partition overlap that kernel's tail.  The partition reads only
+  // seq_lens and the block table, which that kernel does not write (the
+  // contract in attn.h); everything else global -- pages, queries, the
+  // workspace -- is touched only after griddepcontrol.wait.
   if (base & 1023u) {  // the layout below needs a 1024-byte aligned base
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) atomicExch(p.status, kErrBounds);
     return;
   }
-  const uint32_t q_slot = 2u * p.q_half;
+  const uint32_t q_slot = (uint32_t)C::KB * p.q_box;
   const uint32_t nqs = (uint32_t)p.q_slots, nst = (uint32_t)p.stages;
   const uint32_t s_q = base;                       // query slots
-  const uint32_t s_ring = base + nqs * q_slot;     // stages x 32 KB
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw + nqs * q_slot + nst * kStageBytes);
+  const uint32_t s_ring = base + nqs * q_slot;     // stages of C::STAGE bytes
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw + nqs * q_slot + nst * C::STAGE);
   if (tid == 0) {
     for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
@@ -352,10 +416,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     fence_mbarrier_init();
   }
   if (warp == 5) {
-    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_alloc(&sm.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int sl0 = lane < p.B ? p.seq_lens[lane] : 0;
   const int sl1 = lane + 32 < p.B ? p.seq_lens[lane + 32] : 0;
   // Total pages T of the batch and this CTA's share.  Every warp sums the
@@ -373,9 +436,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   T *= p.Hkv;
   const long long G = split_ctas(T, gridDim.x);
   const int c = blockIdx.x;
-  // The combine launch may start now: it waits for this grid's completion
-  // (griddepcontrol.wait) before it reads any partial.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const bool idle = T == 0 || c >= G;
   const long long lo = idle ? 0 : c * T / G, hi = idle ? 0 : (c + 1) * T / G;
   if (warp == 4 && !idle) {
@@ -386,11 +446,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (pg < s0.P)
       asm volatile("prefetch.global.L1 [%0];" ::"l"(p.block_table + (size_t)s0.b * p.max_pages + pg));
   }
+  // The kernel before this one has completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The combine launch may start now: it waits for this grid's completion
+  // (griddepcontrol.wait) before it reads any partial.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (idle) {  // no pages for this CTA
-    if (warp == 5) tmem_dealloc(sm.tmem_base, kTmemCols);
+    if (warp == 5) tmem_dealloc(sm.tmem_base, C::TMEM_COLS);
     return;
   }
   const uint32_t tmem = sm.tmem_base;
@@ -403,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
     if (warp == 5) {
       tc_fence_after();
-      tmem_dealloc(tmem, kTmemCols);
+      tmem_dealloc(tmem, C::TMEM_COLS);
     }
   };
 
@@ -426,9 +491,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const uint32_t qs = n_q % nqs;
         if (n_q >= nqs) ok = mbar_wait(&sm.q_empty[qs], ((n_q / nqs) - 1) & 1, g);
         if (ok) {
-          mbar_arrive_expect_tx(&sm.q_full[qs], 2u * p.rows * 128u);
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(s_q + qs * q_slot + h * p.q_half, &tm_q, &sm.q_full[qs], h * 64,
+          mbar_arrive_expect_tx(&sm.q_full[qs], (uint32_t)C::KB * p.rows * 128u);
+          for (int h = 0; h < C::KB; ++h)
+            tma_load_2d(s_q + qs * q_slot + h * p.q_box, &tm_q, &sm.q_full[qs], h * 64,
                         (b * p.Hq + kvh * p.group) * p.q_len);
         }
       }
@@ -454,15 +519,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const uint32_t st = n_blk % nst;
             if (n_blk >= nst) ok = mbar_wait(&sm.kv_empty[st], ((n_blk / nst) - 1) & 1, g);
             if (ok) {
-              mbar_arrive_expect_tx(&sm.kv_full[st], (uint32_t)nv * 4u * kPageHalf);
-              const uint32_t dst = s_ring + st * kStageBytes;
+              mbar_arrive_expect_tx(&sm.kv_full[st], (uint32_t)nv * (C::KB + C::VB) * kPageBox);
+              const uint32_t dst = s_ring + st * C::STAGE;
               for (int i = 0; i < nv; ++i) {
                 const int tok = pid[i] * kPage;
-                const uint32_t d = dst + i * kPageHalf;
-                tma_load_3d_evict_first(d, &tm_k, &sm.kv_full[st], 0, kvh, tok, pol);
-                tma_load_3d_evict_first(d + kHalf, &tm_k, &sm.kv_full[st], 64, kvh, tok, pol);
-                tma_load_3d_evict_first(d + 2 * kHalf, &tm_v, &sm.kv_full[st], 0, kvh, tok, pol);
-                tma_load_3d_evict_first(d + 3 * kHalf, &tm_v, &sm.kv_full[st], 64, kvh, tok, pol);
+                const uint32_t d = dst + i * kPageBox;
+#pragma unroll
+                for (int h = 0; h < C::KB; ++h)
+                  tma_load_3d_evict_first(d + h * kBox, &tm_k, &sm.kv_full[st], h * 64, kvh, tok, pol);
+#pragma unroll
+                for (int h = 0; h < C::VB; ++h)
+                  tma_load_3d_evict_first(d + (C::KB + h) * kBox, &tm_v, &sm.kv_full[st], h * 64, kvh, tok, pol);
               }
             }
           }
@@ -487,28 +554,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       bool ok = true;
       auto tS = [&](uint32_t gb) { return tmem + ((gb & 1) ? kTmS1 : kTmS0); };
       // S = Q K^T for block gb (nv pages): both operands K-major; k-step kk
-      // starts 32 bytes further into the 128-byte rows, the second 64
-      // features one half further on.
+      // starts 32 bytes further into the 128-byte rows, every 64 features one
+      // box further on.
       auto issue_s = [&](uint32_t gb, uint32_t q_addr, int nv) {
-        const uint32_t stage = s_ring + (gb % nst) * kStageBytes;
+        const uint32_t stage = s_ring + (gb % nst) * C::STAGE;
         const uint64_t a0 = sw128_desc(q_addr, 16, 1024);
         const uint64_t b0 = sw128_desc(stage, 16, 1024);
         const uint32_t idesc = make_idesc(1u, 128, nv * kPage, false);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < DQK / 16; ++kk) {
           const uint32_t bk = kk * 32;
-          const uint32_t offa = ((bk / 128) * p.q_half + (bk % 128)) >> 4;
-          const uint32_t offb = ((bk / 128) * kHalf + (bk % 128)) >> 4;
+          const uint32_t offa = ((bk / 128) * p.q_box + (bk % 128)) >> 4;
+          const uint32_t offb = ((bk / 128) * kBox + (bk % 128)) >> 4;
           mma_f16_ss(tS(gb), a0 + offa, b0 + offb, idesc, kk > 0);
         }
       };
       // O (+)= P V: P from TMEM over S (16 tokens = 8 columns per k-step), V
-      // MN-major with its two 64-feature halves kHalf apart.
-      auto issue_pv = [&](uint32_t gb, int nv, bool acc) {
-        const uint32_t stage = s_ring + (gb % nst) * kStageBytes;
-        const uint64_t b0 = sw128_desc(stage + 2 * kHalf, kHalf, 1024);
+      // MN-major with its 64-feature boxes kBox apart.
+      // a_col = kFineCol: the residual of P in a fine segment.
+      auto issue_pv = [&](uint32_t gb, int nv, bool acc, uint32_t a_col) {
+        const uint32_t stage = s_ring + (gb % nst) * C::STAGE;
+        const uint64_t b0 = sw128_desc(stage + C::KB * kBox, kBox, 1024);
         for (int kk = 0; kk < nv; ++kk)
-          mma_f16_ts(tmem + kTmO, tS(gb) + kk * 8, b0 + ((kk * kPageHalf) >> 4), kIdescPV,
+          mma_f16_ts(tmem + kTmO, tS(gb) + a_col + kk * 8, b0 + ((kk * kPageBox) >> 4), C::IDESC_PV,
                      (acc || kk > 0) ? 1u : 0u);
       };
       while (seg.more() && ok) {
@@ -516,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         long long pre;
         seg.take(b, kvh, pg_lo, pg_hi, pre, P);
         const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
+        const bool fine = seg_fine(P, p.q_len);
         const uint32_t qs = n_q % nqs;
         ok = mbar_wait(&sm.q_full[qs], (n_q / nqs) & 1, g);
         if (!ok) break;
@@ -552,7 +621,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (!ok) break;
           }
           tc_fence_after();
-          issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0);
+          issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0, 0);
+          if (__builtin_expect(fine, 0)) issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), true, kFineCol);
           tc_commit(&sm.kv_empty[gb % nst]);
           tc_commit(&sm.pv_done);
           if (has_next && !s_first) {
@@ -589,6 +659,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       seg.take(b, kvh, pg_lo, pg_hi, pre, P);
       const int len = len_of(p.seq_lens, p.max_pages, b);
       const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
+      const bool fine = seg_fine(P, p.q_len);
       // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
       // the MMA multiplies (normalises o so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
@@ -633,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
-          for (int c4 = 0; c4 < kD / 32; ++c4) {
+          for (int c4 = 0; c4 < DV / 32; ++c4) {
             uint32_t raw[32];
             tmem_ld32(tmem + kTmO + lane_off + c4 * 32, raw);
 #pragma unroll
@@ -662,6 +733,44 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           pk[q2] = bb;
           rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(bb << 16), __uint_as_float(bb & 0xFFFF0000u)));
         }
+        if (__builtin_expect(!fine, 1)) {
+          tmem_st32(tS, pk);
+        } else {
+          // The two-part product: S is still in TMEM (P has not gone over it
+          // yet); P is recomputed exactly as above, rounded (as pk) and its
+          // rounding residual stored to columns kFineCol on.  Kept out of the
+          // loop above, whose registers and schedule it would otherwise change.
+          tmem_ld64(tS, sr);
+          if (seen < kBlkTok) {
+#pragma unroll
+            for (int i = 0; i < kBlkTok; ++i)
+              if (i >= seen) sr[i] = 0xFF800000u;  // -inf
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < kBlkTok / 16; ++c8) {  // 8 pairs (TMEM columns) at a time
+            uint32_t hi8[8], lo8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int q2 = c8 * 8 + i;
+              const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
+              float p0, p1;
+              if ((q2 & 7) >= 6) {
+                f2_split(exp2_poly2(x2), p0, p1);
+              } else {
+                float x0, x1;
+                f2_split(x2, x0, x1);
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              hi8[i] = pack_bf16x2(p0, p1);
+              const float h0 = __uint_as_float(hi8[i] << 16), h1 = __uint_as_float(hi8[i] & 0xFFFF0000u);
+              lo8[i] = pack_bf16x2(p0 - h0, p1 - h1);  // P - h is exact in fp32
+              rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(lo8[i] << 16), __uint_as_float(lo8[i] & 0xFFFF0000u)));
+            }
+            tmem_st8(tS + c8 * 8, hi8);
+            tmem_st8(tS + kFineCol + c8 * 8, lo8);
+          }
+        }
         {
           const uint64_t a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
           const uint64_t bq = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
@@ -671,16 +780,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           l_run += a0 + a1;
           l_rnd += b0 + b1;
         }
-        tmem_st32(tS, pk);
         if (warp == 0 && valid < nv * kPage) {
           // Tokens past the end of the sequence inside its last page: P is 0
           // there, but the cache slots may hold anything (0 * NaN = NaN), so
           // their V rows are cleared before the MMA reads them.
-          const uint32_t vst = s_ring + (gb % nst) * kStageBytes + 2 * kHalf;
+          const uint32_t vst = s_ring + (gb % nst) * C::STAGE + C::KB * kBox;
           const int nrow = nv * kPage - valid;  // rows valid .. nv*16-1 of the block
-          for (int e = lane; e < nrow * 2 * 8; e += 32) {
-            const int row = valid + e / 16, h = (e / 8) & 1, ch = e & 7;
-            const uint32_t a = vst + h * kHalf + row * 128 + ch * 16;
+          for (int e = lane; e < nrow * C::VB * 8; e += 32) {
+            const int row = valid + e / (8 * C::VB), h = (e / 8) % C::VB, ch = e & 7;
+            const uint32_t a = vst + h * kBox + row * 128 + ch * 16;
             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -703,11 +811,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const size_t rec = (((size_t)b * p.Hq + kvh * p.group) * p.q_len + r) * p.max_segs + sidx;
       const float inv = l_rnd > 0.f ? 1.f / l_rnd : 0.f;
 #pragma unroll 1
-      for (int c4 = 0; c4 < kD / 32; ++c4) {
+      for (int c4 = 0; c4 < DV / 32; ++c4) {
         uint32_t raw[32];
         tmem_ld32(tmem + kTmO + lane_off + c4 * 32, raw);
         if (write) {
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * kD + c4 * 32);
+          float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * DV + c4 * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(raw[4 * i]) * inv, __uint_as_float(raw[4 * i + 1]) * inv,
@@ -742,11 +850,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 // The pool [num_pages * 16 tokens, Hkv, D] bf16 as a 3-D tensor, box = one
 // page of one K/V head, 64 features (128 bytes, 128-byte swizzle).
-bool encode_pool(CUtensorMap* map, const void* pool, int num_pages, int Hkv) {
+bool encode_pool(CUtensorMap* map, const void* pool, int num_pages, int Hkv, int D) {
   auto enc = encoder();
   if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)Hkv, (cuuint64_t)num_pages * kPage};
-  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)Hkv * kD * 2};
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)num_pages * kPage};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)kPage};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides, box, estr,
@@ -754,11 +862,11 @@ bool encode_pool(CUtensorMap* map, const void* pool, int num_pages, int Hkv) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 // q [B * Hq rows, D] bf16, box = `box_rows` rows x 64 features (128-byte swizzle).
-bool encode_q(CUtensorMap* map, const void* q, int rows, int box_rows) {
+bool encode_q(CUtensorMap* map, const void* q, int rows, int box_rows, int D) {
   auto enc = encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
@@ -766,42 +874,50 @@ bool encode_q(CUtensorMap* map, const void* q, int rows, int box_rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
 
-int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.D != kD || a.page_size != kPage) return -2;
+template <int DQK, int DV>
+int run_decode(const DecodeArgs& a, cudaStream_t stream) {
+  using C = DecCfg<DQK, DV>;
   const int group = a.Hq / a.Hkv;
   const int q_len = a.q_len > 0 ? a.q_len : 1;
   const int rows = group * q_len;  // query rows per (sequence, K/V head) tile
   if (rows > kMaxGroup) return -2;
   const int max_pages = a.max_pages > 0 ? a.max_pages : 1;
   const int max_segs = decode_max_segments(max_pages);
-  const int q_half = (rows + 7) / 8 * 8 * 128;
-  int q_slots = 1, stages = 2;  // fits for every tile size (static_assert above)
-  if (two_fit(dec_smem_bytes(q_half, 2, 3))) {
-    q_slots = 2;
-    stages = 3;
-  } else if (two_fit(dec_smem_bytes(q_half, 1, 3))) {
-    stages = 3;
-  } else if (two_fit(dec_smem_bytes(q_half, 2, 2))) {
-    q_slots = 2;
+  const int q_box = (rows + 7) / 8 * 8 * 128;
+  // Layout: as many CTAs per SM as the TMEM holds if some layout fits that
+  // many, deepest ring first, then a second query slot; else one per SM.
+  int ctas = 1, q_slots = 1, stages = 2;
+  bool chosen = false;
+  for (int n = C::TMEM_CTAS; n >= 1 && !chosen; --n) {
+    const int cand[4][2] = {{2, 3}, {1, 3}, {2, 2}, {1, 2}};  // (query slots, stages)
+    for (int i = 0; i < 4 && !chosen; ++i) {
+      if (fits(dec_smem_bytes<DQK, DV>(q_box, cand[i][0], cand[i][1]), n)) {
+        ctas = n;
+        q_slots = cand[i][0];
+        stages = cand[i][1];
+        chosen = true;
+      }
+    }
   }
-  int smem = dec_smem_bytes(q_half, q_slots, stages);
-  if (smem < kMinSmem) smem = kMinSmem;
+  if (!chosen) return -2;  // not reached: every width fits once (static_assert)
+  int smem = dec_smem_bytes<DQK, DV>(q_box, q_slots, stages);
+  const int min_smem = kSmemPerSm / (ctas + 1) - 1024 + 16;  // no extra CTA may share the SM
+  if (smem < min_smem) smem = min_smem;
   static int attr_smem[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail_cuda("cudaGetDevice", err);
   if (dev >= 64 || attr_smem[dev] < smem) {
-    err = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    err = cudaFuncSetAttribute(decode_split_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return fail_cuda("decode: cudaFuncSetAttribute", err);
     if (dev < 64) attr_smem[dev] = smem;
   }
   float* ws_o = static_cast<float*>(a.workspace);
-  float* ws_lse = ws_o + (size_t)a.B * a.Hq * q_len * max_segs * kD;
+  float* ws_lse = ws_o + (size_t)a.B * a.Hq * q_len * max_segs * DV;
   int* status = device_status_word();
   if (!status) return fail_cuda("decode: status word", cudaGetLastError());
-  const int split_grid = kCtasPerSm * sm_count();
+  const int split_grid = ctas * sm_count();
   const bool has_pool = a.num_pages > 0 && a.max_pages > 0;
   if (has_pool) {
     SplitParams sp{};
@@ -818,7 +934,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sp.max_segs = max_segs;
     sp.q_len = q_len;
     sp.rows = rows;
-    sp.q_half = q_half;
+    sp.q_box = q_box;
     sp.q_slots = q_slots;
     sp.stages = stages;
     sp.sm_warps = (rows + 31) / 32;
@@ -828,8 +944,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sp.timeout_ns = wait_timeout_ns();
     sp.stall = (debug_flags() & 2) ? 1 : 0;
     CUtensorMap tq, tk, tv;
-    if (!encode_q(&tq, a.q, a.B * a.Hq * q_len, rows) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv) ||
-        !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv))
+    if (!encode_q(&tq, a.q, a.B * a.Hq * q_len, rows, DQK) || !encode_pool(&tk, a.k_pages, a.num_pages, a.Hkv, DQK) ||
+        !encode_pool(&tv, a.v_pages, a.num_pages, a.Hkv, DV))
       return fail_cuda("decode: tensor map", cudaErrorInvalidValue);
     cudaLaunchConfig_t scfg{};
     scfg.gridDim = dim3(split_grid);
@@ -841,7 +957,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     sattr[0].val.programmaticStreamSerializationAllowed = 1;
     scfg.attrs = sattr;
     scfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&scfg, decode_split_kernel, tq, tk, tv, sp);
+    err = cudaLaunchKernelEx(&scfg, decode_split_kernel<DQK, DV>, tq, tk, tv, sp);
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return fail_cuda("decode: split launch", err);
   }
@@ -873,9 +989,33 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, decode_combine_kernel, cp);
+  err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<DV>, cp);
   if (err == cudaSuccess) err = cudaGetLastError();
   return err == cudaSuccess ? 0 : fail_cuda("decode: combine launch", err);
+}
+
+template <int DQK>
+int run_decode_dv(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.Dv) {
+    case 64: return run_decode<DQK, 64>(a, stream);
+    case 128: return run_decode<DQK, 128>(a, stream);
+    case 192: return run_decode<DQK, 192>(a, stream);
+    case 256: return run_decode<DQK, 256>(a, stream);
+    default: return -2;
+  }
+}
+
+}  // namespace
+
+int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.page_size != kPage) return -2;
+  switch (a.D) {
+    case 64: return run_decode_dv<64>(a, stream);
+    case 128: return run_decode_dv<128>(a, stream);
+    case 192: return run_decode_dv<192>(a, stream);
+    case 256: return run_decode_dv<256>(a, stream);
+    default: return -2;
+  }
 }
 
 }  // namespace attn

@@ -54,6 +54,7 @@ struct DecodeArgs {
   void* workspace;
   size_t workspace_bytes;
   int q_len;  // new tokens per sequence (queries), the last q_len cached ones
+  int Dv = 0;  // value width (0: D); D is the query/key width
 };
 
 // Device status word of the current device (nullptr on failure).
@@ -71,7 +72,7 @@ int fail_invalid(const char* msg);
 // Checks of the decode arguments, workspace excepted (attn_api.cu).
 int validate_decode(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
                     const int* seq_lens, const void* o, const float* lse, int B, int Hq, int Hkv, int q_len, int D,
-                    int page_size, int num_pages, int max_pages_per_seq, float scale);
+                    int Dv, int page_size, int num_pages, int max_pages_per_seq, float scale);
 
 // Launchers: return a status code of include/attn.h.
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
@@ -114,7 +115,7 @@ inline int decode_max_segments(int max_pages) {
   return (max_pages + kDecodeMinChunk - 1) / kDecodeMinChunk + 1;
 }
 // Workspace: partial outputs [B*Hq][S][D] f32 and their log2-sum-exp
-// [B*Hq][S] f32, S = segments.
+// [B*Hq][S] f32, S = segments (D: the value width).
 inline size_t decode_workspace_bytes(int B, int Hq, int max_pages, int D) {
   const size_t rows = (size_t)B * Hq, segs = (size_t)decode_max_segments(max_pages);
   return rows * segs * (size_t)(D + 1) * 4;

@@ -102,12 +102,20 @@ constexpr int kEmuPairsPer8 = FP8 ? ATTN_EMU_PAIRS_PER8_FP8 : ATTN_EMU_PAIRS_PER
 constexpr bool kSplitP = ATTN_SPLIT_P != 0;
 constexpr int kSplitKeys = ATTN_SPLIT_P * 16;
 static_assert(ATTN_SPLIT_P == 0 || (ATTN_SPLIT_P % 2 == 0 && ATTN_SPLIT_P < 8), "split at 32, 64 or 96 keys");
-// bf16 path: O is normalised by the sum of the bf16-rounded P that the MMA
-// multiplies (1) or by the exact fp32 row sum (0).  On rows of a few keys the
-// two sums differ by up to 2^-10, which with the bf16 rounding of O can exceed
-// 1e-2 absolute.  The e4m3 path always uses the rounded sum.
+// Which sum normalises O.  The MMA multiplies V by P rounded to bf16 / e4m3,
+// so normalising by the sum of those rounded values makes the weights add to
+// exactly one; normalising by the exact fp32 sum (which the LSE needs anyway)
+// is off by the mean rounding error of the row's weights: up to 2^-9 / 2^-4
+// relative on a row of a few keys -- with the bf16 rounding of O beyond 1e-2
+// for bf16 -- but ~2^-9 / sqrt(n) (bf16) or ~2^-4 / sqrt(n) (e4m3) on a row of
+// n keys, since round-to-nearest errors are unbiased.  The kernels built for
+// tiles whose rows see few keys (FINE) keep the rounded sum (3-4 instructions
+// per key pair) and normalise fine tiles by it; other tiles, whose rows see
+// >= 256 (bf16) or >= 512 (e4m3) keys, use the exact sum in every kernel: 2e-4
+// and 3e-3 of |O| typically.
+// ATTN_ROUNDED_SUM=1 keeps the rounded sum everywhere (measurement switch).
 #ifndef ATTN_ROUNDED_SUM
-#define ATTN_ROUNDED_SUM 1
+#define ATTN_ROUNDED_SUM 0
 #endif
 static_assert(ATTN_ROUNDED_SUM == 0 || ATTN_ROUNDED_SUM == 1, "row-sum mode 0 or 1");
 
@@ -723,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + (t == 0 ? C::TM_S0 : C::TM_S1) + lane_off;
     const uint32_t tO = tmem + (t == 0 ? C::TM_O0 : C::TM_O1) + lane_off;
     const float sl2 = p.scale_log2;
-    constexpr bool kRsum = FP8 || ATTN_ROUNDED_SUM;
+    constexpr bool kRsum = FINE || ATTN_ROUNDED_SUM;
     uint32_t scnt = 0, nunit = 0;
     bool ok = true;
     for (int rnd = 0, u = unit_of(0, p.n_units); u < p.n_units && ok; u = unit_of(++rnd, p.n_units)) {
@@ -845,7 +853,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm.st_m[t][r] = m_run - shift;  // P carried 2^shift: LSE = m - shift + log2(sum)
         sm.st_l[t][r] = l_run;
-        sm.st_r[t][r] = kRsum ? l_rnd : l_run;
+        // rounded sum on fine tiles only: the other tiles of a FINE kernel
+        // then agree bit for bit with the kernel built without it
+        sm.st_r[t][r] = (kRsum && (fine || ATTN_ROUNDED_SUM)) ? l_rnd : l_run;
         mbar_arrive(&sm.st_full[t]);
         ++nunit;
       }

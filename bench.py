@@ -32,8 +32,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import (FP8_CAUSAL, GQA_CAUSAL, MQA_DECODE, SWA_CAUSAL, decode_inputs, decode_queries,  # noqa: E402
-                       prefill_inputs, prefill_inputs_fp8, seed_of)
+from workloads import (FP8_CAUSAL, GQA_CAUSAL, LATENT_192_128, LATENT_256, MQA_DECODE, SWA_CAUSAL,  # noqa: E402
+                       DecodeShape, decode_inputs, decode_queries, prefill_inputs, prefill_inputs_fp8, seed_of)
 from workloads.accounting import decode_bytes, prefill_bytes, prefill_flops  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (prefill) & decode HBM GB/s, % of B200 roofline"
@@ -41,14 +41,14 @@ PREFILL = GQA_CAUSAL
 DECODE = MQA_DECODE
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# the ncu captures summarised under profiles/, valid only for the kernel
-# sources they were taken on (sha256 prefix of the files); a changed kernel
-# reports null until it is captured again.
+# an ncu capture of the kernel, valid only for the kernel sources it was taken
+# on (sha256 prefix of the files); a changed kernel reports null until it is
+# captured again.
 PROFILED_TRAFFIC = {
     "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "9e739ca46748c6ba",
-                "bytes": 361_058_560 + 97_935_616, "profile": "profiles/prefill_gqa_causal_B4_H32_L4096_D128.md"},
+                "bytes": 361_058_560 + 97_935_616},
     "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "bc446ec70993fe26",
-               "bytes": 147_640_832 + 4_014_848, "profile": "profiles/decode_mqa_paged_B64_H32_D128.md"},
+               "bytes": 147_640_832 + 4_014_848},
 }
 
 
@@ -62,12 +62,19 @@ def profiled_traffic(kernel: str):
     return entry["bytes"] if h.hexdigest()[:16] == entry["sha"] else None
 L2_FLUSH_BYTES = 256 << 20
 DECODE_LAYERS = 3  # K/V pools decoded per step
+E2E_MAX_STEPS = 50  # the end-to-end loop copies ~490 MB per step: at most this many steps
+SIDE_MIN_MS = 120.0  # each side measurement runs launches for at least this long (clock samples)
+SUSTAINED_S = 2.0  # length of the sustained-clock prefill loop
+# MQA decode in a 256-wide latent space: the decode workload's batch, lengths
+# and layout with D = 256 (a side line; 285 MB of K/V)
+LATENT_DECODE = DecodeShape("latent_mqa_paged_decode_B64_H32_Hkv1_D256_len512_8192", B=64, Hq=32, Hkv=1, D=256,
+                            len_lo=512, len_hi=8192)
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' side measurements")
@@ -122,7 +129,7 @@ def measured_peaks():
 class ClockSampler:
     """Samples the SM clock and the throttle reasons of the GPU under test
     from a background thread while the timed region runs: through NVML every
-    5 ms, so that a region of a few tens of milliseconds still gets samples,
+    millisecond, so that a region of ten milliseconds still gets ten samples,
     else with nvidia-smi every 200 ms.  Only samples taken between
     ``begin()`` and ``end()`` (host time around the region, whose GPU work
     the final synchronize bounds) are reported.  The device is matched by
@@ -170,7 +177,7 @@ class ClockSampler:
             r = get_reasons(h)
             self.rows.append((t, float(sm), float(mx), {self.REASONS[i] for i in range(4) if r & bits[i]}))
             self._first.set()
-            self._stop.wait(0.005)
+            self._stop.wait(0.001)
 
     def _poll_smi(self):
         while not self._stop.is_set():
@@ -197,7 +204,7 @@ class ClockSampler:
     def _run(self):
         try:
             pynvml, h = self._nvml_handle()
-            self.source = "nvml, 5 ms"
+            self.source = "nvml, 1 ms"
             self._poll_nvml(pynvml, h)
         except Exception:
             self.source = "nvidia-smi, 200 ms"
@@ -400,21 +407,26 @@ def run_ours(args):
 
     e2e_step()
     torch.cuda.synchronize()
+    K_e2e = min(K, E2E_MAX_STEPS)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(K):
+    for _ in range(K_e2e):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = world * pf * K / (e2e_ms / 1e3) / 1e12
+    e2e_value = world * pf * K_e2e / (e2e_ms / 1e3) / 1e12
+
+    # ---- the prefill alone, back to back for SUSTAINED_S seconds: the figure
+    # at the clock a long run settles to (the timed region above is shorter)
+    sustained = sustained_prefill(attn, q, k, v, o, lse, stream, gpu_uuid, local, world, dev, pf, peaks)
 
     # ---- side measurements of the other workloads (not part of the step)
     extra = {}
     if not args.no_extra:
-        extra = side_workloads(attn, dev, peaks, world)
+        extra = side_workloads(attn, dev, peaks, world, gpu_uuid, local)
 
     cpu = None
     if rank == 0 and world == 1:
@@ -467,8 +479,13 @@ def run_ours(args):
                          "timing": "the first pool's call alone, after the L2 flush, events around it"},
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": (1 + 2 * DECODE_LAYERS) * K,  # prefill + (split, combine) per decode call
+                "d2h_bytes_per_step": d2h, "steps": K_e2e},
+        "prefill_sustained": sustained,
+        # per step: the prefill's two launches (its leading row groups, whose
+        # rows see fewer than 256 keys, run in the kernel built with the
+        # two-part P V product; the rest in the other) + (split, combine) per
+        # decode call
+        "gpu_launches": (2 + 2 * DECODE_LAYERS) * K,
         "clocks": clk,
         "cpu_baseline": cpu,
         "workloads": extra,
@@ -510,58 +527,146 @@ def fp8_gemm_peak(dev):
         return None
 
 
-def side_workloads(attn, dev, peaks, world):
-    """Per-launch TFLOP/s of the sliding-window and FP8 workloads (median of
-    5 launches after 2 warm-ups; inputs larger than L2)."""
+def side_timer(fn, dev, world, gpu_uuid, local, min_ms=SIDE_MIN_MS, before=None):
+    """Times one launch sequence ``fn`` on the current stream: 2 warm-ups,
+    then launches with CUDA events around each (``before`` runs untimed ahead
+    of each, e.g. an L2 flush) until at least ``min_ms`` of host time and 5
+    launches have passed, with SM clocks sampled meanwhile.  Returns the median
+    ms per launch (max over ranks) and the clock record."""
+    import torch
+    for _ in range(2):
+        if before:
+            before()
+        fn()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_uuid, local)
+    clocks.start()
+    clocks.begin()
+    ts = []
+    t0 = time.perf_counter()
+    while len(ts) < 5 or (time.perf_counter() - t0) * 1e3 < min_ms:
+        if before:
+            before()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    clocks.end()
+    clk = clocks.stop()
+    clk["launches"] = len(ts)
+    return max_over_ranks(statistics.median(ts), world, dev), clk
+
+
+def sustained_prefill(attn, q, k, v, o, lse, stream, gpu_uuid, local, world, dev, pf, peaks):
+    """The GQA causal prefill back to back for SUSTAINED_S seconds (one event
+    pair around the whole loop, clocks sampled): TFLOP/s at the clock a long
+    run settles to, against the sustained bf16 peak."""
+    import torch
+    n = 0
+    clocks = ClockSampler(gpu_uuid, local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    clocks.begin()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < SUSTAINED_S:
+        for _ in range(20):
+            attn.attn_fwd(q, k, v, PREFILL.scale, PREFILL.causal, PREFILL.window, o=o, lse=lse)
+        n += 20
+        if n % 200 == 0:
+            torch.cuda.synchronize()
+    b.record(stream)
+    torch.cuda.synchronize()
+    clocks.end()
+    clk = clocks.stop()
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / n
+    tf = pf / (ms / 1e3) / 1e12
+    return {"TFLOP/s": round(tf, 1), "ms_per_launch": round(ms, 4), "launches": n,
+            "frac_of_sustained_peak": round(tf / peaks["bf16_tflops_sustained"], 4),
+            "frac_of_burst_peak": round(tf / peaks["bf16_tflops"], 4), "clocks": clk}
+
+
+def side_workloads(attn, dev, peaks, world, gpu_uuid="", local=0):
+    """Per-launch throughput of the other workloads, each timed by side_timer
+    (inputs larger than L2) with its own clock record."""
     import torch
     out = {}
-    for shape, idx in ((SWA_CAUSAL, 3), (FP8_CAUSAL, 4)):
-        if shape.fp8:
-            q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, seed_of(idx))
+    T = lambda fn, **kw: side_timer(fn, dev, world, gpu_uuid, local, **kw)  # noqa: E731
+    fp8_peak = fp8_gemm_peak(dev)
+    for shape, idx, fmt in ((SWA_CAUSAL, 3, None), (FP8_CAUSAL, 4, "e4m3"), (FP8_CAUSAL, 4, "e5m2"),
+                            (LATENT_192_128, 1, None), (LATENT_256, 3, None)):
+        if fmt:
+            q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, seed_of(idx), fmt=fmt)
             q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
-            fn = lambda: attn.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, shape.scale, shape.causal, shape.window)  # noqa
+            call = attn.attn_fwd_fp8 if fmt == "e4m3" else attn.attn_fwd_e5m2
+            fn = lambda: call(q8, k8, v8, sq, sk, sv, shape.scale, shape.causal, shape.window)  # noqa
         else:
             q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(idx))]
-            fn = lambda: attn.attn_fwd(q, k, v, shape.scale, shape.causal, shape.window)  # noqa
-        for _ in range(2):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(5):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ms = max_over_ranks(statistics.median(ts), world, dev)
+            call = attn.attn_fwd_mla if shape.dv != 128 or shape.D != 128 else attn.attn_fwd
+            fn = lambda: call(q, k, v, shape.scale, shape.causal, shape.window)  # noqa
+        ms, clk = T(fn)
         tf = prefill_flops(shape) / (ms / 1e3) / 1e12
         entry = {"TFLOP/s": round(tf, 1), "ms": round(ms, 3), "bytes_MB": round(prefill_bytes(shape) / 1e6, 1)}
-        if shape.fp8:
+        if fmt:
             entry["frac_of_bf16_peak"] = round(tf / peaks["bf16_tflops"], 4)
-            fp8_peak = fp8_gemm_peak(dev)
             if fp8_peak:
                 entry["fp8_peak_tflops"] = round(fp8_peak, 1)
                 entry["frac_of_fp8_peak"] = round(tf / fp8_peak, 4)
-                entry["fp8_peak_source"] = "measured here: cuBLASLt e4m3 8192^3 GEMM (torch._scaled_mm), best of 10"
+                entry["fp8_peak_source"] = ("measured here: cuBLASLt e4m3 8192^3 GEMM (torch._scaled_mm), best of 10"
+                                            + ("; the dense 8-bit tensor rate, e5m2 included" if fmt == "e5m2" else ""))
             else:
                 entry["note"] = "FP8 GEMM probe unavailable; nominal dense FP8 is 2x bf16"
         else:
             entry["frac"] = round(tf / peaks["bf16_tflops"], 4)
-        out[shape.name] = entry
+        entry["clocks"] = clk
+        out[shape.name + ("_e5m2" if fmt == "e5m2" else "")] = entry
         del fn
         torch.cuda.empty_cache()
-    out.update(multi_token_decode(attn, dev, peaks, world))
-    out.update(paged_chunk_prefill(attn, dev, peaks, world))
-    out.update(backward_pass(attn, dev, peaks, world))
+    out.update(multi_token_decode(attn, dev, peaks, world, T))
+    out.update(latent_decode(attn, dev, peaks, world, T))
+    out.update(paged_chunk_prefill(attn, dev, peaks, world, T))
+    out.update(backward_pass(attn, dev, peaks, world, T))
     return out
 
 
-def backward_pass(attn, dev, peaks, world):
+def latent_decode(attn, dev, peaks, world, T):
+    """GB/s of the MQA paged decode with D = 256 (the decode workload's batch
+    and lengths, 285 MB of K/V), L2 flushed (write, then read 256 MB) before
+    each call."""
+    import torch
+    sh = LATENT_DECODE
+    kv = decode_inputs(sh, seed_of(2))
+    d = {n: getattr(kv, n).to(dev) for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+    o = torch.empty_like(d["q"])
+    lse = torch.empty(d["q"].shape[:2], dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.attn_decode_workspace_bytes(sh.B, sh.Hq, kv.max_pages, sh.D), dtype=torch.uint8,
+                     device=dev)
+    fw = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fr = torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        fw.zero_()
+        fr.view(torch.int32).sum(dtype=torch.int32)
+
+    fn = lambda: attn.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],  # noqa
+                                        sh.scale, o=o, lse=lse, workspace=ws)
+    ms, clk = T(fn, before=flush)
+    by = decode_bytes(sh, kv.seq_lens.tolist())
+    gbs = by / (ms / 1e3) / 1e9
+    return {sh.name: {"GB/s": round(gbs, 1), "us_per_call": round(ms * 1e3, 2),
+                      "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes_MB": round(by / 1e6, 1),
+                      "timing": "alone after an L2 flush", "clocks": clk}}
+
+
+def backward_pass(attn, dev, peaks, world, T):
     """attn_bwd on the GQA causal prefill workload (its own forward's O and
     LSE): 5 products of the visible (query, key) pairs against the forward's
-    2, i.e. 2.5x the forward's FLOPs.  Median of 5 after 2 warm-ups; the
-    inputs (201 MB) and the dQ accumulator (272 MB) exceed L2."""
+    2, i.e. 2.5x the forward's FLOPs.  The inputs (201 MB) and the dQ
+    accumulator (272 MB) exceed L2."""
     import torch
     shape = PREFILL
     q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(1))]
@@ -573,30 +678,18 @@ def backward_pass(attn, dev, peaks, world):
                      device=dev)
     fn = lambda: attn.attn_bwd(q, k, v, o, do, lse, shape.scale, shape.causal, shape.window,  # noqa: E731
                                dq=dq, dk=dk, dv=dv, workspace=ws)
-    for _ in range(2):
-        fn()
-    torch.cuda.synchronize()
-    ts = []
-    for _ in range(5):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        fn()
-        b.record()
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    ms = max_over_ranks(statistics.median(ts), world, dev)
+    ms, clk = T(fn)
     tf = 2.5 * prefill_flops(shape) / (ms / 1e3) / 1e12
     return {f"backward_{shape.name}": {"TFLOP/s": round(tf, 1), "ms": round(ms, 3),
-                                       "frac": round(tf / peaks["bf16_tflops"], 4)}}
+                                       "frac": round(tf / peaks["bf16_tflops"], 4), "clocks": clk}}
 
 
-def paged_chunk_prefill(attn, dev, peaks, world, B=4, Hq=32, Hkv=8, D=128, cached=3072, chunk=1024):
+def paged_chunk_prefill(attn, dev, peaks, world, T, B=4, Hq=32, Hkv=8, D=128, cached=3072, chunk=1024):
     """Chunked prefill over a paged cache (attn_prefill_paged): each of B
     sequences holds `cached` tokens plus a `chunk` of new ones, 16-token pages
     in a permuted pool; the chunk attends causally to all of them.  Also the
-    KV append of the chunk (attn_kv_append).  Median of 5 after 2 warm-ups."""
+    KV append of the chunk (attn_kv_append)."""
     import torch
-    from workloads import DecodeShape
     shape = DecodeShape("paged_chunk", B=B, Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=1)
     L = cached + chunk
     kv = decode_inputs(shape, seed_of(1) + 200, seq_lens=[L] * B)
@@ -607,35 +700,21 @@ def paged_chunk_prefill(attn, dev, peaks, world, B=4, Hq=32, Hkv=8, D=128, cache
     v_new = torch.randn(B, Hkv, chunk, D, generator=g).to(torch.bfloat16).to(dev)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-
-    def timed(fn):
-        for _ in range(2):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(5):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return max_over_ranks(statistics.median(ts), world, dev)
-
-    ms = timed(lambda: attn.attn_prefill_paged(q, kp, vp, bt, sl, shape.scale, o=o, lse=lse))
+    ms, clk = T(lambda: attn.attn_prefill_paged(q, kp, vp, bt, sl, shape.scale, o=o, lse=lse))
     flops = 4.0 * D * Hq * B * (chunk * cached + chunk * (chunk + 1) / 2)
     tf = flops / (ms / 1e3) / 1e12
-    ms_app = timed(lambda: attn.attn_kv_append(k_new, v_new, kp, vp, bt, sl))
+    ms_app, clk_app = T(lambda: attn.attn_kv_append(k_new, v_new, kp, vp, bt, sl))
     app_bytes = 2 * 2 * B * Hkv * chunk * D * 2  # K and V, read and written
     return {f"paged_chunk_prefill_B{B}_H{Hq}_G{Hq // Hkv}_cached{cached}_chunk{chunk}_D{D}": {
-        "TFLOP/s": round(tf, 1), "ms": round(ms, 3), "frac": round(tf / peaks["bf16_tflops"], 4),
-        "kv_append_GB/s": round(app_bytes / (ms_app / 1e3) / 1e9, 1), "kv_append_us": round(ms_app * 1e3, 2)}}
+        "TFLOP/s": round(tf, 1), "ms": round(ms, 3), "frac": round(tf / peaks["bf16_tflops"], 4), "clocks": clk,
+        "kv_append_GB/s": round(app_bytes / (ms_app / 1e3) / 1e9, 1), "kv_append_us": round(ms_app * 1e3, 2),
+        "kv_append_clocks": clk_app}}
 
 
-def multi_token_decode(attn, dev, peaks, world, q_len: int = 4):
+def multi_token_decode(attn, dev, peaks, world, T, q_len: int = 4):
     """GB/s of the batch-64 MQA decode with q_len new tokens per sequence
     (attn_decode_paged_multi): every page read once for all q_len tokens.
-    L2 flushed (write, then read 256 MB) before each call; median of 10."""
+    L2 flushed (write, then read 256 MB) before each call."""
     import torch
     kv = decode_inputs(DECODE, seed_of(2))
     qm = decode_queries(DECODE, q_len, seed_of(2) + 100).to(dev)
@@ -646,26 +725,18 @@ def multi_token_decode(attn, dev, peaks, world, q_len: int = 4):
                      dtype=torch.uint8, device=dev)
     fw = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     fr = torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    fn = lambda: attn.attn_decode_paged_multi(qm, kp, vp, bt, sl, DECODE.scale, o=o, lse=lse, workspace=ws)  # noqa
-    for _ in range(3):
-        fn()
-    torch.cuda.synchronize()
-    ts = []
-    for _ in range(10):
+
+    def flush():
         fw.zero_()
         fr.view(torch.int32).sum(dtype=torch.int32)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        fn()
-        b.record()
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    ms = max_over_ranks(statistics.median(ts), world, dev)
+
+    fn = lambda: attn.attn_decode_paged_multi(qm, kp, vp, bt, sl, DECODE.scale, o=o, lse=lse, workspace=ws)  # noqa
+    ms, clk = T(fn, before=flush)
     by = decode_bytes(DECODE, kv.seq_lens.tolist(), q_len)
     gbs = by / (ms / 1e3) / 1e9
     return {f"{DECODE.name}_qlen{q_len}": {"GB/s": round(gbs, 1), "us_per_call": round(ms * 1e3, 2),
                                             "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                                            "bytes_MB": round(by / 1e6, 1)}}
+                                            "bytes_MB": round(by / 1e6, 1), "clocks": clk}}
 
 
 # ------------------------------------------------------------- reference

@@ -15,8 +15,10 @@
  *                             held in fixed-size pages addressed through a
  *                             block table, split over the cache and merged by
  *                             log-sum-exp (attn_decode_paged_multi: the last
- *                             q_len cached tokens; attn_decode_paged_noalloc:
- *                             scratch inside the library).
+ *                             q_len cached tokens; attn_decode_paged_mla: keys
+ *                             and values of different widths;
+ *                             attn_decode_paged_noalloc: scratch inside the
+ *                             library).
  *   attn_prefill_paged        a chunk of new tokens against the paged cache
  *                             (chunked prefill), with attn_kv_append writing
  *                             the chunk's K/V into its pages.
@@ -47,9 +49,13 @@
  *   - All launches are asynchronous on the caller's CUDA stream `stream`
  *     (a cudaStream_t passed as void*; NULL = legacy default stream).
  *     The decode kernels are launched as programmatic dependents of the
- *     kernel before them in the stream: they may become resident and set up
- *     early, but read and write no global memory until that kernel has
- *     completed, so stream order holds as for a plain launch.
+ *     kernel before them in the stream: they may become resident, set up and
+ *     read seq_lens and block_table early, while that kernel still runs;
+ *     queries, pages, the workspace and the outputs are read or written only
+ *     after it has completed.  So the kernel immediately before a decode call
+ *     (attn_decode_paged*) in the same stream must not write that call's
+ *     seq_lens or block_table; with any other operation between them (a copy,
+ *     an event, another kernel) stream order holds as for a plain launch.
  *   - A call returns ATTN_OK once its kernels are enqueued.  Argument errors
  *     are detected on the host before anything is launched and return
  *     ATTN_ERR_INVALID / ATTN_ERR_UNSUPPORTED with nothing written.  A CUDA
@@ -217,8 +223,8 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
  * attn_decode_workspace_bytes -- size of the scratch buffer attn_decode_paged
  * needs for these sizes: per query head of every sequence, up to
  * S = ceil(max_pages_per_seq / 32) + 1 partial results of D + 1 floats
- * (B * Hq * S * (D + 1) * 4 bytes).  Host only; never fails (0 for empty
- * shapes).
+ * (B * Hq * S * (D + 1) * 4 bytes; D is the value width).  Host only; never
+ * fails (0 for empty shapes).
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq, int D);
 
@@ -245,8 +251,8 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int max_pages_per_seq
  * bottom-right corner); cache slots past seq_lens[b] in a sequence's last
  * page are never used, whatever they hold.  seq_lens[b] == 0 gives O = 0 and
  * LSE = -inf.
- * Supported: page_size == 16, D == 128, Hq % Hkv == 0 and Hq / Hkv <= 128
- * (otherwise ATTN_ERR_UNSUPPORTED).
+ * Supported: page_size == 16, D in {64, 128, 192, 256}, Hq % Hkv == 0 and
+ * Hq / Hkv <= 128 (otherwise ATTN_ERR_UNSUPPORTED).
  * Page ids are trusted unless bounds-check mode is on (attn_set_debug), in
  * which case an id outside [0, num_pages) reads as a page of zeros and is
  * reported as ATTN_ERR_BOUNDS by attn_last_device_error().  Pages are copied
@@ -285,6 +291,31 @@ ATTN_API int attn_decode_paged_multi(const void* q, const void* k_pages, const v
                                      int B, int Hq, int Hkv, int q_len, int D, int page_size, int num_pages,
                                      int max_pages_per_seq, float scale,
                                      void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_decode_paged_mla -- attn_decode_paged_multi with keys and values of
+ * different widths: queries and keys of width D_qk, values of width D_v,
+ * attention in a latent space (latent projection of the page "高效多头潜在
+ * 注意力解码技术：Flash MLA深度解析", §2.1) against a paged cache.
+ *
+ *   q        [B, Hq, q_len, D_qk] bf16: the last q_len cached tokens
+ *   k_pages  [num_pages, page_size, Hkv, D_qk] bf16
+ *   v_pages  [num_pages, page_size, Hkv, D_v] bf16 (same page ids as k_pages)
+ *   o        [B, Hq, q_len, D_v] bf16 (written); lse [B, Hq, q_len] fp32
+ *            (written; may be NULL)
+ *   workspace  at least attn_decode_workspace_bytes(B, Hq * q_len,
+ *              max_pages_per_seq, D_v) bytes
+ *   everything else as attn_decode_paged_multi.
+ *
+ * Supported: D_qk, D_v in {64, 128, 192, 256}, page_size == 16,
+ * (Hq / Hkv) * q_len <= 128 (otherwise ATTN_ERR_UNSUPPORTED).  With
+ * D_v > 128 the tensor memory holds one decode CTA per SM instead of two.
+ */
+ATTN_API int attn_decode_paged_mla(const void* q, const void* k_pages, const void* v_pages,
+                                   const int* block_table, const int* seq_lens, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int q_len, int D_qk, int D_v,
+                                   int page_size, int num_pages, int max_pages_per_seq, float scale,
+                                   void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * attn_prefill_paged -- chunked prefill over a paged KV cache: the last Lq

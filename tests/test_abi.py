@@ -124,7 +124,7 @@ def _dec(cdll, **kw):
     (dict(sl=_P(0)), -1),
     (dict(bt=_P(0x10002)), -1),         # misaligned int32 table
     (dict(page=32), -2),                # only 16-token pages are built
-    (dict(D=64), -2),
+    (dict(D=96), -2),                   # widths 64, 128, 192, 256 are built
     (dict(Hq=256, Hkv=1), -2),          # group > 128
     (dict(B=0), 0),
 ])

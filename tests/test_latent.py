@@ -118,3 +118,78 @@ def test_latent_rejects_unsupported_widths(lib):
     with pytest.raises(lib.AttnError) as e:
         lib.attn_fwd_mla(q, q, v)
     assert e.value.status == lib.ATTN_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ decode
+from workloads import DecodeShape, decode_inputs, decode_queries  # noqa: E402
+
+
+def _decode_case(lens, Hq, Hkv, D, Dv, seed, nan_tail=False):
+    shape = DecodeShape("ld", B=len(lens), Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=1, Dv=Dv)
+    kv = decode_inputs(shape, seed, seq_lens=lens, extra_pages=3)
+    if nan_tail:
+        for b, n in enumerate(lens):
+            npg = (n + 15) // 16
+            if npg and n % 16:
+                last = int(kv.block_table[b, npg - 1])
+                kv.k_pages[last, n % 16:] = float("nan")
+                kv.v_pages[last, n % 16:] = float("nan")
+    return shape, kv
+
+
+@pytest.mark.parametrize("D", [64, 192, 256])
+@pytest.mark.parametrize("lens,Hq,Hkv", [
+    ([1, 15, 16, 17, 512, 513, 3000, 0], 32, 1),
+    ([3, 100, 1000, 2049], 32, 4),
+    ([50, 33, 16], 12, 4),               # group of 3
+    ([300, 77], 128, 1),                 # four softmax warps
+])
+def test_decode_widths(lib, D, lens, Hq, Hkv):
+    """attn_decode_paged at head widths other than 128."""
+    shape, kv = _decode_case(lens, Hq, Hkv, D, D, 60 + D + sum(lens), nan_tail=True)
+    d = {n: getattr(kv, n).cuda() for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+    o, lse = lib.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], shape.scale)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, lse, o_ref, l_ref, f"decode D={D} {lens}")
+
+
+@pytest.mark.parametrize("dqk,dv", [(192, 128), (256, 128), (128, 256), (64, 192), (256, 256), (128, 64)])
+@pytest.mark.parametrize("lens,Hq,Hkv,q_len", [
+    ([100, 17, 1, 2000, 0], 32, 1, 1),
+    ([50, 3, 700, 4096], 32, 8, 4),
+    ([513, 64], 12, 4, 7),
+])
+def test_decode_latent_widths(lib, dqk, dv, lens, Hq, Hkv, q_len):
+    """attn_decode_paged_mla: keys of width D_qk, values of width D_v, one or
+    several new tokens per sequence, NaN in the unused slots of last pages."""
+    shape, kv = _decode_case(lens, Hq, Hkv, dqk, dv, 70 + dqk + dv + q_len, nan_tail=True)
+    q = decode_queries(shape, q_len, 71 + q_len)
+    d = {n: getattr(kv, n).cuda() for n in ("k_pages", "v_pages", "block_table", "seq_lens")}
+    o, lse = lib.attn_decode_paged_mla(q.cuda(), d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                       shape.scale)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    assert o.shape == (len(lens), Hq, q_len, dv)
+    o_ref, l_ref = oracle.paged_decode(q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    _check(o, lse, o_ref, l_ref, f"decode {dqk}/{dv} {lens} q_len={q_len}")
+
+
+LATENT_DECODE = DecodeShape("latent_mqa_paged_decode_B64_H32_Hkv1_D256_len512_8192", B=64, Hq=32, Hkv=1, D=256,
+                            len_lo=512, len_hi=8192)
+
+
+def test_decode_latent_full_workload(lib):
+    """MQA decode in a 256-wide latent space: the batch-64 paged decode
+    workload's lengths and layout with D = 256, every row against the
+    oracle."""
+    kv = decode_inputs(LATENT_DECODE, seed_of(2))
+    d = {n: getattr(kv, n).cuda() for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+    o, lse = lib.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                   LATENT_DECODE.scale)
+    torch.cuda.synchronize()
+    assert lib.attn_last_device_error() == 0
+    o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens,
+                                       LATENT_DECODE.scale)
+    _check(o, lse, o_ref, l_ref, LATENT_DECODE.name)

@@ -291,6 +291,28 @@ def test_paged_decode_equals_contiguous_definition():
         np.testing.assert_allclose(lse[b], lb[0, :, 0], rtol=0, atol=1e-13)
 
 
+def test_paged_decode_values_of_another_width():
+    """Keys of width 8 and values of width 5 (latent shapes): each sequence's
+    result is the scalar brute force over its gathered cache, one query token
+    and the last three (bottom-right causal)."""
+    shape = DecodeShape("w", B=3, Hq=4, Hkv=2, D=8, len_lo=1, len_hi=40, Dv=5)
+    kv = decode_inputs(shape, 52, seq_lens=[3, 17, 31], extra_pages=2)
+    assert kv.v_pages.shape[-1] == 5
+    q3 = torch.randn(3, 4, 3, 8, generator=torch.Generator().manual_seed(53)).to(torch.bfloat16)
+    for q, multi in ((kv.q, False), (q3, True)):
+        o, lse = oracle.paged_decode(q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, 0.3)
+        for b, n in enumerate(kv.seq_lens.tolist()):
+            npg = (n + 15) // 16
+            ids = kv.block_table[b, :npg].long()
+            kb = kv.k_pages[ids].reshape(npg * 16, 2, 8)[:n].permute(1, 0, 2)
+            vb = kv.v_pages[ids].reshape(npg * 16, 2, 5)[:n].permute(1, 0, 2)
+            qb = (q[b][None] if multi else q[b][None, :, None]).double().numpy()
+            ob, lb = _brute(qb, kb[None].double().numpy(), vb[None].double().numpy(), 0.3, multi, 0)
+            got_o, got_l = (o[b], lse[b]) if multi else (o[b][:, None], lse[b][:, None])
+            np.testing.assert_allclose(got_o, ob[0], rtol=0, atol=1e-13)
+            np.testing.assert_allclose(got_l, lb[0], rtol=0, atol=1e-13)
+
+
 def test_paged_decode_invariant_to_page_permutation():
     """Re-scatter the pages to new pool slots and permute the block table to
     match: the result must not change (PagedAttention section of p3)."""

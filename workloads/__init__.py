@@ -71,10 +71,15 @@ class DecodeShape:
     len_lo: int
     len_hi: int
     page_size: int = PAGE_SIZE
+    Dv: int = 0              # value width; 0 = D (queries and keys have width D)
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.D)
+
+    @property
+    def dv(self) -> int:
+        return self.Dv or self.D
 
 
 # The five workloads of the build, indexed 0..4.  The seed of workload i is
@@ -160,7 +165,7 @@ def prefill_inputs_fp8(shape: PrefillShape, seed: int, fmt: str = "e4m3"):
 class PagedKV:
     q: torch.Tensor            # [B, Hq, D] bf16
     k_pages: torch.Tensor      # [num_pages, page_size, Hkv, D] bf16
-    v_pages: torch.Tensor      # [num_pages, page_size, Hkv, D] bf16
+    v_pages: torch.Tensor      # [num_pages, page_size, Hkv, Dv] bf16
     block_table: torch.Tensor  # [B, max_pages] int32
     seq_lens: torch.Tensor     # [B] int32
 
@@ -193,7 +198,7 @@ def decode_inputs(shape: DecodeShape, seed: int, seq_lens: Optional[list] = None
     need = sum(pages_per_seq)
     num_pages = max(1, need + extra_pages)
     k_pages = _normal(g, (num_pages, ps, shape.Hkv, shape.D)).to(torch.bfloat16)
-    v_pages = _normal(g, (num_pages, ps, shape.Hkv, shape.D)).to(torch.bfloat16)
+    v_pages = _normal(g, (num_pages, ps, shape.Hkv, shape.dv)).to(torch.bfloat16)
     perm = torch.randperm(num_pages, generator=g).to(torch.int32)
     table = torch.zeros((shape.B, max_pages), dtype=torch.int32)
     cursor = 0
