@@ -88,8 +88,13 @@ constexpr float kLn2 = 0.6931471805599453f;
 #ifndef ATTN_EMU_PAIRS_PER8
 #define ATTN_EMU_PAIRS_PER8 0
 #endif
+// e4m3: 1 of 8.  Without the rounded row sum (plain tiles) its softmax issues
+// ~7 instructions per key pair but waits 16 MUFU cycles for the two ex2, so
+// one polynomial pair in 8 moves work to idle issue slots (interleaved A/B on
+// the e4m3 workload: 1,449 against 1,387 TFLOP/s; 2 and 3 of 8: 1,391, 1,368).
+// bf16, MUFU-bound no more than its tensor work, measured best with none.
 #ifndef ATTN_EMU_PAIRS_PER8_FP8
-#define ATTN_EMU_PAIRS_PER8_FP8 0
+#define ATTN_EMU_PAIRS_PER8_FP8 1
 #endif
 template <bool FP8>
 constexpr int kEmuPairsPer8 = FP8 ? ATTN_EMU_PAIRS_PER8_FP8 : ATTN_EMU_PAIRS_PER8;
@@ -297,13 +302,14 @@ static_assert(sizeof(Smem) <= 4096, "barrier/statistics block exceeds its reserv
 // FINE (8-bit P only): also the residual fp8(P - h) into pk_lo, and the sum
 // of h + residual, the weight the two products apply together.  E5M2: P and
 // its residual in e5m2 (the format of e5m2 inputs), else e4m3.
-template <bool FP8, bool RSUM, bool FINE, bool E5M2 = false>
+// EMU: of every 8 pairs, this many take the FMA-pipe polynomial for 2^x.
+template <bool FP8, bool RSUM, bool FINE, bool E5M2 = false, int EMU = 0>
 __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2,
                                        uint64_t (&rs2)[4], uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2],
                                        uint32_t (&pk_lo)[kBN / 2]) {
   const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
   float p0, p1;
-  if ((q2 & 7) >= 8 - kEmuPairsPer8<FP8>) {
+  if ((q2 & 7) >= 8 - EMU) {
     f2_split(exp2_poly2(x2), p0, p1);
   } else {
     float x0, x1;
@@ -343,11 +349,11 @@ __device__ __forceinline__ void p_pair(int q2, const uint32_t (&sr)[kBN], uint64
   }
 }
 
-template <bool FP8, bool RSUM, bool FINE, int Q_LO, int Q_HI, bool E5M2 = false>
+template <bool FP8, bool RSUM, bool FINE, int Q_LO, int Q_HI, bool E5M2 = false, int EMU = 0>
 __device__ __forceinline__ void p_pairs(const uint32_t (&sr)[kBN], uint64_t sc2, uint64_t nm2, uint64_t (&rs2)[4],
                                         uint64_t (&rr2)[4], uint32_t (&pk)[kBN / 2], uint32_t (&pk_lo)[kBN / 2]) {
 #pragma unroll
-  for (int q2 = Q_LO; q2 < Q_HI; ++q2) p_pair<FP8, RSUM, FINE, E5M2>(q2, sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+  for (int q2 = Q_LO; q2 < Q_HI; ++q2) p_pair<FP8, RSUM, FINE, E5M2, EMU>(q2, sr, sc2, nm2, rs2, rr2, pk, pk_lo);
 }
 
 // Fine tiles: pairs [Q_LO, Q_HI) in chunks of 8 TMEM columns (e4m3: 16 pairs,
@@ -812,7 +818,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (fine) {
               p_pairs_fine<FP8, kRsum, E5M2, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
             } else {
-              p_pairs<FP8, kRsum, false, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo);
+              // (the exponent polynomial only in the kernels for plain tiles)
+              p_pairs<FP8, kRsum, false, Q_LO, Q_HI, false, FINE ? 0 : kEmuPairsPer8<FP8>>(sr, sc2, nm2, rs2, rr2,
+                                                                                           pk, pk_lo);
               tmem_st_cols<C0, C1>(tS, pk);
             }
           };

@@ -21,6 +21,7 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -45,10 +46,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # on (sha256 prefix of the files); a changed kernel reports null until it is
 # captured again.
 PROFILED_TRAFFIC = {
-    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "9e739ca46748c6ba",
-                "bytes": 361_058_560 + 97_935_616},
-    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "bc446ec70993fe26",
-               "bytes": 147_640_832 + 4_014_848},
+    # the plain prefill launch (rows 256-4095; the 19 us launch of rows 0-255 not included)
+    "prefill": {"files": ["csrc/prefill_sm100.cu", "csrc/sm100_ptx.cuh"], "sha": "0987b1613cc02e1c",
+                "bytes": 360_202_752 + 90_787_840},
+    "decode": {"files": ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"], "sha": "246f5bfa3e7e6ac1",
+               "bytes": 147_637_760 + 3_635_712},
 }
 
 
@@ -79,7 +81,54 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' side measurements")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle baseline")
+    ap.add_argument("--profile", choices=sorted(PROFILE_WORKLOADS), default=None,
+                    help="only launch this workload's kernels warmup + steps times (for profiler captures)")
     return ap.parse_args(argv)
+
+
+# Workloads --profile can launch alone: (shape, seed index, input format or
+# call name).  The FP8 one runs at half the workload's length (a quarter of its
+# work, inputs still 3 x 64 MB > L2) so that a many-pass capture stays short.
+PROFILE_WORKLOADS = {
+    "prefill": (GQA_CAUSAL, 1, "bf16"),
+    "swa": (SWA_CAUSAL, 3, "bf16"),
+    "fp8": (dataclasses.replace(FP8_CAUSAL, name="fp8_causal_B1_H32_L16384_D128", Lq=16384, Lk=16384), 4, "e4m3"),
+    "e5m2": (dataclasses.replace(FP8_CAUSAL, name="fp8_causal_B1_H32_L16384_D128", Lq=16384, Lk=16384), 4, "e5m2"),
+    "latent256": (LATENT_256, 3, "mla"),
+    "decode": (MQA_DECODE, 2, "decode"),
+}
+
+
+def run_profile(args):
+    """Launches one workload's kernels (warmup + steps times) and exits: the
+    command profiler captures run, with nothing else on the device."""
+    import torch
+    import attention_flash_attn_02_b200 as attn
+    attn.load()
+    dev = torch.device("cuda", 0)
+    shape, idx, kind = PROFILE_WORKLOADS[args.profile]
+    if kind == "decode":
+        kv = decode_inputs(shape, seed_of(idx))
+        d = {n: getattr(kv, n).to(dev) for n in ("q", "k_pages", "v_pages", "block_table", "seq_lens")}
+        fn = lambda: attn.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],  # noqa: E731
+                                            d["seq_lens"], shape.scale)
+    elif kind in ("e4m3", "e5m2"):
+        q8, k8, v8, sq, sk, sv = prefill_inputs_fp8(shape, seed_of(idx), fmt=kind)
+        q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+        call = attn.attn_fwd_fp8 if kind == "e4m3" else attn.attn_fwd_e5m2
+        fn = lambda: call(q8, k8, v8, sq, sk, sv, shape.scale, shape.causal, shape.window)  # noqa: E731
+    else:
+        q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(idx))]
+        call = attn.attn_fwd_mla if kind == "mla" else attn.attn_fwd
+        fn = lambda: call(q, k, v, shape.scale, shape.causal, shape.window)  # noqa: E731
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    st = attn.attn_last_device_error()
+    print(json.dumps({"profile": args.profile, "workload": shape.name, "launches": args.warmup + args.steps,
+                      "status": attn.attn_status_str(st)}))
+    if st != 0:
+        sys.exit(1)
 
 
 # ------------------------------------------------------------ distributed
@@ -787,7 +836,9 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
