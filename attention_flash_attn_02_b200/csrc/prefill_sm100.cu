@@ -415,6 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // A launch queued behind this one as a programmatic dependent (the few-key
+  // launch) may start on SMs this grid leaves idle; it shares no data with it.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -462,6 +465,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       tmem_dealloc(tmem, 512);
     }
+    // Launched as a programmatic dependent (the few-key launch after the
+    // plain one): complete only after the launch before it, so that stream
+    // order holds for both.  Without a prerequisite grid this returns at once.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
   };
 
   // Each role branch sets its own register count first thing, so that no code
@@ -959,9 +966,11 @@ int host_key_count(int i, int lk, const PrefillArgs& a) {
   return h - lo;
 }
 
+// dependent: launch as a programmatic dependent of the kernel before it in the
+// stream (it reads nothing that kernel writes, and waits for it before exit).
 template <int D, bool FP8, bool PAGED, bool E5M2, bool FINE>
 int launch_range(const PrefillArgs& a, Params p, int mg_lo, int mg_hi, const CUtensorMap& tq,
-                 const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+                 const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream, bool dependent = false) {
   using C = Cfg<D, FP8, E5M2>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -996,8 +1005,18 @@ int launch_range(const PrefillArgs& a, Params p, int mg_lo, int mg_hi, const CUt
     p.l2_hints = 1;
   }
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
-  prefill_kernel<D, FP8, PAGED, E5M2, FINE><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-  err = cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  err = cudaLaunchKernelEx(&cfg, prefill_kernel<D, FP8, PAGED, E5M2, FINE>, tq, tk, tv, p);
+  if (err == cudaSuccess) err = cudaGetLastError();
   return err == cudaSuccess ? 0 : fail_cuda("prefill: launch", err);
 }
 
@@ -1075,10 +1094,14 @@ int run(const PrefillArgs& a, cudaStream_t stream) {
         if (!any) break;
         ++mg_fine;
       }
+      // The plain launch goes first; the few-key launch follows as its
+      // programmatic dependent, so that its short units fill the SMs the
+      // plain launch's tail leaves idle instead of running on their own.
       int st = 0;
-      if (mg_fine > 0) st = launch_range<D, FP8, PAGED, E5M2, true>(a, p, 0, mg_fine, tq, tk, tv, stream);
-      if (st == 0 && mg_fine < n_mgroups)
+      if (mg_fine < n_mgroups)
         st = launch_range<D, FP8, PAGED, E5M2, false>(a, p, mg_fine, n_mgroups, tq, tk, tv, stream);
+      if (st == 0 && mg_fine > 0)
+        st = launch_range<D, FP8, PAGED, E5M2, true>(a, p, 0, mg_fine, tq, tk, tv, stream, mg_fine < n_mgroups);
       return st;
     }
   }
