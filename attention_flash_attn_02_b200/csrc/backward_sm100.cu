@@ -17,19 +17,27 @@
 //       warp 8       TMA producer: K_j and V_j once, then Q_i and dO_i
 //                    (double buffered) per step.
 //       warp 9       TMEM owner; one thread issues per step
-//                      S^T = K_j Q_i^T  and  dP^T = V_j dO_i^T   (TMEM),
+//                      dP^T = V_j dO_i^T                        (TMEM),
 //                    then, once P^T and dS^T are written back,
 //                      dV += P^T dO_i   and  dK += dS^T Q_i      (A from TMEM)
 //                      dQ_i = dS K_j                            (A from smem)
-//       warps 0-3    one thread per key (TMEM lane): P^T and dS^T of its key
-//                    against the block's 128 queries, back to TMEM as bf16,
-//                    and dS (bf16) into a swizzled shared-memory tile.
-//       warps 4-7    one thread per query row: dQ_i from TMEM added to the
-//                    fp32 accumulator (vector reductions).
+//                    and S^T = K_j Q_{i'}^T of the next step, which runs
+//                    while dQ_i is read out.
+//       warps 0-3    one thread per key (TMEM lane): P^T of its key against
+//                    the block's 128 queries as soon as S^T is there (back to
+//                    TMEM as bf16), then dS^T once dP^T is (back to TMEM, and
+//                    dS (bf16) into a swizzled shared-memory tile).
+//       warps 4-7    one thread per query row: dQ_i from TMEM into a
+//                    128-byte-swizzled fp32 staging tile (the dS tile, free
+//                    between the dQ product and the next step's dS), which
+//                    the TMA unit adds to the fp32 accumulator with bulk
+//                    tensor reductions, 64 features at a time.
 //                    At the end warps 0-3 write dK (times scale) and dV.
 //   bwd_post_kernel   dQ = bf16(scale * accumulator).
-// TMEM (512 columns): [0,128) S^T, then P^T over its first 64, then dQ_i;
-// [128,256) dP^T, then dS^T over its first 64; [256,384) dV; [384,512) dK.
+// TMEM (512 columns): [0,128) S^T, then P^T over its first 64; [128,256)
+// dP^T, then dS^T over its first 64, then dQ_i; [256,384) dV; [384,512) dK.
+// So the next step's S^T can be computed, and its P^T formed, while dQ_i is
+// still being read out; only dP^T waits for the read-out.
 // Every operand tile is a 128-row, 128-byte-swizzled TMA tile, used K-major
 // or MN-major by its descriptor; dS is stored [key][query] so that dQ reads
 // it MN-major.
@@ -92,8 +100,10 @@ struct BParams {
 
 struct BSmem {
   uint64_t kv_full, q_full[2], q_empty[2];
-  uint64_t s_full, p_full, dq_full, dq_empty, ds_empty, fin, drain;
+  uint64_t s_full, dp_full, p_full, dq_full, dq_empty, ds_empty, fin, drain;
   uint64_t stat;  // a step's LSE/Dvec written to shared memory (128 arrivals)
+  uint64_t stg_full;  // dQ staging written (128 arrivals, per 64-feature half)
+  uint64_t stg_free;  // ... and read by the bulk reduction (1 arrival)
   uint32_t tmem_base;
   int abort_flag;
   float lse2[2][kT];  // [buffer][query]
@@ -115,6 +125,9 @@ __device__ __forceinline__ void query_range(const BParams& p, int k0, int k1, in
   r_hi = r_hi > p.Lq ? p.Lq : r_hi;
 }
 
+// The dQ staging (two fp32 boxes of 128 rows x 32 features) reuses the dS tile.
+static_assert(2 * BCfg<128>::BOX_BYTES == BCfg<128>::DS_BYTES, "dQ staging fills the dS tile");
+
 template <int D>
 constexpr bool bwd_fits() {
   return BCfg<D>::SMEM_TILES + (int)sizeof(BSmem) <= BCfg<D>::SMEM_BYTES;
@@ -125,8 +138,9 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BParams p) {
+               const __grid_constant__ CUtensorMap tm_dq, const BParams p) {
   using C = BCfg<D>;
+  constexpr int kDqHalves = D / 64;  // dQ leaves TMEM 64 features (two fp32 boxes) at a time
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   if ((base & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned base
@@ -155,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_empty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.p_full, 128);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_empty, 128);
@@ -162,6 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.fin, 1);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.stat, 128);
+    mbar_init(&sm.stg_full, 128);
+    mbar_init(&sm.stg_free, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -223,27 +240,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dv_desc = sw128_desc(base + C::OFF_V, 16, 1024);   // V_j K-major (dP^T A)
       const uint64_t kmn_desc = sw128_desc(base + C::OFF_K, C::BOX_BYTES, 1024);  // K_j MN-major (dQ B)
       const uint64_t ds_desc = sw128_desc(base + C::OFF_DS, C::BOX_BYTES, 1024);  // dS MN-major (dQ A)
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const int qs = s & 1;
-        ok = mbar_wait(&sm.q_full[qs], (s >> 1) & 1, g);
-        if (!ok) break;
-        if (s > 0) {  // S^T's columns hold the previous dQ until it has been read
-          ok = mbar_wait(&sm.dq_empty, (s - 1) & 1, g);
-          if (!ok) break;
-        }
-        tc_fence_after();
-        const uint32_t q_tile = base + C::OFF_Q + qs * C::TILE_BYTES;
-        const uint32_t do_tile = base + C::OFF_DO + qs * C::TILE_BYTES;
-        const uint64_t q_km = sw128_desc(q_tile, 16, 1024), do_km = sw128_desc(do_tile, 16, 1024);
-        // S^T = K_j Q_i^T and dP^T = V_j dO_i^T, k-steps of 16 features
+      // S^T = K_j Q_i^T of step s into TM_S, k-steps of 16 features
+      auto issue_st = [&](int s) {
+        const uint64_t q_km = sw128_desc(base + C::OFF_Q + (s & 1) * C::TILE_BYTES, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t bk = kk * 32;
           const uint32_t off = ((bk / 128) * C::BOX_BYTES + (bk % 128)) >> 4;
           mma_f16_ss(tmem + C::TM_S, dk_desc + off, q_km + off, C::ID_S, kk > 0);
-          mma_f16_ss(tmem + C::TM_DP, dv_desc + off, do_km + off, C::ID_S, kk > 0);
         }
         tc_commit(&sm.s_full);
+      };
+      if (ok) ok = mbar_wait(&sm.q_full[0], 0, g);
+      if (ok) {
+        tc_fence_after();
+        issue_st(0);
+      }
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int qs = s & 1;
+        if (s > 0) {  // dP^T's columns hold the previous dQ until it has been read
+          ok = mbar_wait(&sm.dq_empty, (s - 1) & 1, g);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint32_t q_tile = base + C::OFF_Q + qs * C::TILE_BYTES;
+        const uint32_t do_tile = base + C::OFF_DO + qs * C::TILE_BYTES;
+        const uint64_t do_km = sw128_desc(do_tile, 16, 1024);
+        // dP^T = V_j dO_i^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t bk = kk * 32;
+          const uint32_t off = ((bk / 128) * C::BOX_BYTES + (bk % 128)) >> 4;
+          mma_f16_ss(tmem + C::TM_DP, dv_desc + off, do_km + off, C::ID_S, kk > 0);
+        }
+        tc_commit(&sm.dp_full);
         ok = mbar_wait(&sm.p_full, s & 1, g);
         if (!ok) break;
         tc_fence_after();
@@ -257,15 +287,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f16_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, do_mn + off, C::ID_ACC, (s > 0 || kk > 0) ? 1u : 0u);
           mma_f16_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, q_mn + off, C::ID_ACC, (s > 0 || kk > 0) ? 1u : 0u);
         }
-        // dQ_i = dS K_j over the tile's 128 keys (both operands MN-major)
+        // dQ_i = dS K_j over the tile's 128 keys (both operands MN-major),
+        // into the dP^T columns: issued after dK, their last reader
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk) {
           const uint32_t off = (kk * 16 * 128) >> 4;
-          mma_f16_ss(tmem + C::TM_S, ds_desc + off, kmn_desc + off, C::ID_DQ, kk > 0);
+          mma_f16_ss(tmem + C::TM_DP, ds_desc + off, kmn_desc + off, C::ID_DQ, kk > 0);
         }
         tc_commit(&sm.dq_full);
         tc_commit(&sm.q_empty[qs]);
         tc_commit(&sm.ds_empty);
+        // The next step's S^T: its columns' last reader (dV, P^T) was issued
+        // above, and MMAs run in issue order.
+        if (s + 1 < nsteps) {
+          ok = mbar_wait(&sm.q_full[(s + 1) & 1], ((s + 1) >> 1) & 1, g);
+          if (!ok) break;
+          tc_fence_after();
+          issue_st(s + 1);
+        }
       }
       tc_commit(&sm.fin);  // dK and dV complete
       tc_commit(&sm.drain);
@@ -280,57 +319,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int off = p.Lk - p.Lq;
     bool ok = true;
+    // LSE (log2) and Dvec of query r of step s's block; each thread loads one
+    // of the 128 and shares it through shared memory.
+    auto load_stat = [&](int s, float& l2v, float& dvv) {
+      const int q = step_blk(s) * kT + r;
+      const size_t row = (size_t)(b * p.Hq + step_head(s)) * p.Lq + q;
+      l2v = q < p.Lq ? p.lse2[row] : INFINITY;
+      dvv = q < p.Lq ? p.dvec[row] : 0.f;
+    };
+    // All 128 values of step s are in place once every thread has arrived on
+    // `stat` (an mbarrier, so the wait is bounded).  Step s + 1's values go
+    // into the other buffer once step s's softmax is done, which is also
+    // after every thread is done with step s - 1, the buffer's last user.
+    auto put_stat = [&](int s, float l2v, float dvv) {
+      sm.lse2[s & 1][r] = l2v;
+      sm.dvec[s & 1][r] = dvv;
+      mbar_arrive(&sm.stat);
+    };
+    if (nsteps > 0) {
+      float l2v, dvv;
+      load_stat(0, l2v, dvv);
+      put_stat(0, l2v, dvv);
+    }
+    // visible queries of this key: q + off >= key (causal), q + off - W + 1 <= key (window)
+    const int q_first = p.causal ? key - off : INT_MIN;
+    const int q_last = (p.causal && p.window > 0) ? key - off + p.window - 1 : INT_MAX;
+    const bool key_ok = key < p.Lk;
     for (int s = 0; s < nsteps && ok; ++s) {
-      const int h = step_head(s), i = step_blk(s);
-      const int bh = b * p.Hq + h;
+      const int i = step_blk(s);
       const int buf = s & 1;
-      {  // this block's LSE (log2) and Dvec into shared memory, one per thread
-        const int q = i * kT + r;
-        const size_t row = (size_t)bh * p.Lq + q;
-        sm.lse2[buf][r] = q < p.Lq ? p.lse2[row] : INFINITY;
-        sm.dvec[buf][r] = q < p.Lq ? p.dvec[row] : 0.f;
-        // All 128 values of this step are in place once every thread has
-        // arrived (an mbarrier, so the wait is bounded).  A thread arrives
-        // for step s only after it is done with step s - 1, whose buffer
-        // step s + 1 reuses.
-        mbar_arrive(&sm.stat);
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.stat, s & 1, g));
-        if (!ok) break;
-      }
+      float nl2 = INFINITY, ndv = 0.f;  // the next step's values, loaded early
+      if (s + 1 < nsteps) load_stat(s + 1, nl2, ndv);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.stat, s & 1, g));
+      if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full, s & 1, g));
       if (!ok) break;
-      if (s > 0) {  // the dS tile is free once the previous dQ MMA has read it
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.ds_empty, (s - 1) & 1, g));
-        if (!ok) break;
-      }
       tc_fence_after();
-      // visible queries of this key: q + off >= key (causal), q + off - W + 1 <= key (window)
-      const int q_first = p.causal ? key - off : INT_MIN;
-      const int q_last = (p.causal && p.window > 0) ? key - off + p.window - 1 : INT_MAX;
-      const bool key_ok = key < p.Lk;
-#pragma unroll 1
+      // P^T from S^T (masked entries 0), back to TMEM as bf16 over S^T's
+      // first 64 columns; the packed values stay for dS.
+      uint32_t pp[kT / 2];
+#pragma unroll
       for (int c = 0; c < kT / 32; ++c) {
-        uint32_t sr[32], dr[32];
+        uint32_t sr[32];
         tmem_ld32(tmem + C::TM_S + lane_off + c * 32, sr);
-        tmem_ld32(tmem + C::TM_DP + lane_off + c * 32, dr);
-        uint32_t pp[16], dd[16];
 #pragma unroll
         for (int t = 0; t < 32; t += 2) {
-          float pv[2], dsv[2];
+          float pv[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int qq = c * 32 + t + e;
             const int q = i * kT + qq;
             const bool vis = key_ok && q >= q_first && q <= q_last;
             const float x = fmaf(__uint_as_float(sr[t + e]), p.scale_log2, -sm.lse2[buf][qq]);
-            const float pe = vis ? ex2_approx(x) : 0.f;
-            pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(dr[t + e]) - sm.dvec[buf][qq]);
+            pv[e] = vis ? ex2_approx(x) : 0.f;
           }
-          pp[t / 2] = pack_bf16x2(pv[0], pv[1]);
-          dd[t / 2] = pack_bf16x2(dsv[0], dsv[1]);
+          pp[c * 16 + t / 2] = pack_bf16x2(pv[0], pv[1]);
         }
-        tmem_st16(tmem + C::TM_S + lane_off + c * 16, pp);
+        tmem_st16(tmem + C::TM_S + lane_off + c * 16, pp + c * 16);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.dp_full, s & 1, g));
+      if (!ok) break;
+      if (s > 0) {  // the dS tile is free once the previous dQ has left its staging
+        const uint32_t n_last = (uint32_t)s * kDqHalves - 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.stg_free, n_last & 1, g));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      // dS = P (dP - Dvec), with P as rounded for the dV product
+#pragma unroll
+      for (int c = 0; c < kT / 32; ++c) {
+        uint32_t dr[32];
+        tmem_ld32(tmem + C::TM_DP + lane_off + c * 32, dr);
+        uint32_t dd[16];
+#pragma unroll
+        for (int t = 0; t < 32; t += 2) {
+          const uint32_t pw = pp[c * 16 + t / 2];
+          const float p0 = __uint_as_float(pw << 16), p1 = __uint_as_float(pw & 0xFFFF0000u);
+          const int qq = c * 32 + t;
+          dd[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dr[t]) - sm.dvec[buf][qq]),
+                                  p1 * (__uint_as_float(dr[t + 1]) - sm.dvec[buf][qq + 1]));
+        }
         tmem_st16(tmem + C::TM_DP + lane_off + c * 16, dd);
         // dS row (queries c*32 .. c*32+31 of key r) into the swizzled tile:
         // 64-query boxes, 16-byte chunks XORed with the row's low 3 bits
@@ -347,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // dS visible to the tensor core
       tc_fence_before();
       mbar_arrive(&sm.p_full);
+      if (s + 1 < nsteps) put_stat(s + 1, nl2, ndv);
     }
     // dK (times scale) and dV of this key row
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.fin, 0, g));
@@ -386,27 +455,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ dQ_i into the accumulator
     const int r = (warp & 3) * 32 + lane;  // query row of the block = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const bool leader = threadIdx.x == 4 * 32;  // issues the bulk reductions
+    const uint32_t stage = base + C::OFF_DS;    // two 32-feature fp32 boxes of BOX_BYTES (16 KB)
+    uint32_t n_use = 0;                         // staging uses so far
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, s & 1, g));
       if (!ok) break;
       tc_fence_after();
-      const int q = step_blk(s) * kT + r;
-      float* dst = p.dq_acc + ((size_t)(b * p.Hq + step_head(s)) * p.Lq + q) * D;
+      const int bh = b * p.Hq + step_head(s), r0 = step_blk(s) * kT;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + C::TM_S + lane_off + c * 32, v);
-        if (q < p.Lq) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            red_add_v4(dst + c * 32 + 4 * u, __uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                       __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+      for (int h = 0; h < kDqHalves && ok; ++h, ++n_use) {
+        uint32_t v[64];
+        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        if (h == kDqHalves - 1) {  // TMEM read out: the next dP^T may go there
+          tc_fence_before();
+          mbar_arrive(&sm.dq_empty);
         }
+        if (n_use > 0) {  // the staging tile's previous contents have been read
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.stg_free, (n_use - 1) & 1, g));
+          if (!ok) break;
+        }
+        // row r of both boxes: 8 chunks of 16 bytes each, XOR-swizzled by the
+        // row's low 3 bits (the 128-byte swizzle of the reduction's tensor map)
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t a = stage + bb * C::BOX_BYTES + r * 128 + ((u ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[bb * 32 + 4 * u]),
+                         "r"(v[bb * 32 + 4 * u + 1]), "r"(v[bb * 32 + 4 * u + 2]), "r"(v[bb * 32 + 4 * u + 3])
+                         : "memory");
+          }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging visible to the TMA unit
+        mbar_arrive(&sm.stg_full);
+        if (leader) {
+          ok = mbar_wait(&sm.stg_full, n_use & 1, g);
+          if (ok) {
+            // rows past Lq fall outside the tensor map and are not written
+            tma_reduce_add_3d(&tm_dq, stage, h * 64, r0, bh);
+            tma_reduce_add_3d(&tm_dq, stage + C::BOX_BYTES, h * 64 + 32, r0, bh);
+            bulk_commit_group();
+            bulk_wait_read_all();
+            mbar_arrive(&sm.stg_free);
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
       }
-      tc_fence_before();
-      mbar_arrive(&sm.dq_empty);
     }
+    if (leader) bulk_wait_all();  // every reduction has completed
     finish();
   } else {
     finish();  // warps 10-11
@@ -461,6 +559,20 @@ PFN_cuTensorMapEncodeTiled_v12000 bwd_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   }
   return fn;
+}
+
+// The fp32 dQ accumulator [outer, rows, D] as a 3-D tensor, box 32 features x
+// 128 rows (128 bytes a row, 128-byte swizzle), the target of bulk reductions.
+bool bwd_encode_acc(CUtensorMap* map, void* base, int D, uint64_t rows, uint64_t outer) {
+  auto enc = bwd_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, rows, outer};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)D * 4 * rows};
+  cuuint32_t box[3] = {32, (cuuint32_t)kT, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // [outer, rows, D] bf16, box 64 features x 128 rows (128-byte swizzle).
@@ -518,13 +630,14 @@ int run_bwd(const BackwardArgs& a, cudaStream_t stream) {
     p.status = device_status_word();
     if (!p.status) return fail_cuda("backward: status word", cudaGetLastError());
     p.timeout_ns = wait_timeout_ns();
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if (!bwd_encode(&tq, a.q, D, a.Lq, (uint64_t)a.B * a.Hq) ||
         !bwd_encode(&tdo, a.dout, D, a.Lq, (uint64_t)a.B * a.Hq) ||
-        !bwd_encode(&tk, a.k, D, a.Lk, (uint64_t)a.B * a.Hkv) || !bwd_encode(&tv, a.v, D, a.Lk, (uint64_t)a.B * a.Hkv))
+        !bwd_encode(&tk, a.k, D, a.Lk, (uint64_t)a.B * a.Hkv) || !bwd_encode(&tv, a.v, D, a.Lk, (uint64_t)a.B * a.Hkv) ||
+        !bwd_encode_acc(&tdq, dq_acc, D, a.Lq, (uint64_t)a.B * a.Hq))
       return fail_cuda("backward: tensor map", cudaErrorInvalidValue);
     const long long grid = (long long)p.n_kt * a.B * a.Hkv;
-    bwd_kernel<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    bwd_kernel<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail_cuda("backward: launch", err);
   }
