@@ -358,22 +358,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P^T from S^T (masked entries 0), back to TMEM as bf16 over S^T's
       // first 64 columns; the packed values stay for dS.
       uint32_t pp[kT / 2];
+      // a key that sees every query of the block needs no per-element test
+      // (rows past Lq have LSE +inf, so their P is 0 either way)
+      const bool all_vis = __all_sync(0xffffffffu, key_ok && i * kT >= q_first && i * kT + kT - 1 <= q_last);
 #pragma unroll
       for (int c = 0; c < kT / 32; ++c) {
         uint32_t sr[32];
         tmem_ld32(tmem + C::TM_S + lane_off + c * 32, sr);
+        if (all_vis) {
 #pragma unroll
-        for (int t = 0; t < 32; t += 2) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int qq = c * 32 + t + e;
-            const int q = i * kT + qq;
-            const bool vis = key_ok && q >= q_first && q <= q_last;
-            const float x = fmaf(__uint_as_float(sr[t + e]), p.scale_log2, -sm.lse2[buf][qq]);
-            pv[e] = vis ? ex2_approx(x) : 0.f;
+          for (int t = 0; t < 32; t += 2) {
+            const uint64_t x2 = fma2(f2(__uint_as_float(sr[t]), __uint_as_float(sr[t + 1])),
+                                     f2(p.scale_log2, p.scale_log2),
+                                     f2(-sm.lse2[buf][c * 32 + t], -sm.lse2[buf][c * 32 + t + 1]));
+            float x0, x1;
+            f2_split(x2, x0, x1);
+            pp[c * 16 + t / 2] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
           }
-          pp[c * 16 + t / 2] = pack_bf16x2(pv[0], pv[1]);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; t += 2) {
+            float pv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int qq = c * 32 + t + e;
+              const int q = i * kT + qq;
+              const bool vis = key_ok && q >= q_first && q <= q_last;
+              const float x = fmaf(__uint_as_float(sr[t + e]), p.scale_log2, -sm.lse2[buf][qq]);
+              pv[e] = vis ? ex2_approx(x) : 0.f;
+            }
+            pp[c * 16 + t / 2] = pack_bf16x2(pv[0], pv[1]);
+          }
         }
         tmem_st16(tmem + C::TM_S + lane_off + c * 16, pp + c * 16);
       }
@@ -464,15 +479,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int bh = b * p.Hq + step_head(s), r0 = step_blk(s) * kT;
-#pragma unroll 1
-      for (int h = 0; h < kDqHalves && ok; ++h, ++n_use) {
-        uint32_t v[64];
-        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
-        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        if (h == kDqHalves - 1) {  // TMEM read out: the next dP^T may go there
-          tc_fence_before();
-          mbar_arrive(&sm.dq_empty);
-        }
+      // All of dQ_i out of TMEM first (its columns then take the next dP^T),
+      // then through the staging tile 64 features at a time.
+      uint32_t v[kDqHalves][64];
+#pragma unroll
+      for (int h = 0; h < kDqHalves; ++h) {
+        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v[h]));
+        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v[h] + 32));
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.dq_empty);
+#pragma unroll
+      for (int h = 0; h < kDqHalves; ++h, ++n_use) {
         if (n_use > 0) {  // the staging tile's previous contents have been read
           ok = __all_sync(0xffffffffu, mbar_wait(&sm.stg_free, (n_use - 1) & 1, g));
           if (!ok) break;
@@ -484,8 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const uint32_t a = stage + bb * C::BOX_BYTES + r * 128 + ((u ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[bb * 32 + 4 * u]),
-                         "r"(v[bb * 32 + 4 * u + 1]), "r"(v[bb * 32 + 4 * u + 2]), "r"(v[bb * 32 + 4 * u + 3])
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[h][bb * 32 + 4 * u]),
+                         "r"(v[h][bb * 32 + 4 * u + 1]), "r"(v[h][bb * 32 + 4 * u + 2]), "r"(v[h][bb * 32 + 4 * u + 3])
                          : "memory");
           }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging visible to the TMA unit
