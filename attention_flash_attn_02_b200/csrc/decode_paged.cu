@@ -59,17 +59,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kSmemPerSm = 233472;  // shared memory of an SM, 1 KB of it reserved per CTA
-// Segments of sequences whose first query token sees fewer than kFineKeys
-// cached tokens multiply V by P in two bf16 parts, P rounded and its rounding
-// residual (TMEM columns 32-63 of the S buffer; P of a 64-token block fills
-// 0-31): on a row of a few keys, rounding P to bf16 alone moves O by up to
-// ~2^-9 of the spread of its V values, which with the bf16 rounding of O can
-// pass 1e-2.  Decided from the sequence's page count P, which every role
-// already has (its capacity P * 16 bounds the length): P * 16 - q_len + 1 <
-// kFineKeys.
-constexpr int kFineKeys = 256;
-constexpr uint32_t kFineCol = 32;
-__device__ __forceinline__ bool seg_fine(int pages, int q_len) { return pages * kPage - q_len + 1 < kFineKeys; }
+// Sequences whose first query token sees fewer than kShortKeys cached tokens
+// ("short") take no part in the split kernel's page partition: the combine
+// kernel computes their rows directly in fp32 (exact softmax weights).  On a
+// row of a few keys the tensor-core path's bf16 rounding of P alone moves O
+// by up to ~2^-9 of the spread of its V values, which with the bf16 rounding
+// of O can pass 1e-2; handling those rows elsewhere keeps the split kernel's
+// hot loop free of any extra code (residual-product code there cost 0.5-4 us
+// per call even when no segment used it).
+constexpr int kShortKeys = 256;
+__device__ __forceinline__ bool is_short(int len, int q_len) { return len - q_len + 1 < kShortKeys; }
 
 // Per-width constants: query/key width DQK, value width DV (64..256).
 template <int DQK, int DV>
@@ -152,8 +151,10 @@ __device__ __forceinline__ int len_of(const int* seq_lens, int max_pages, int b)
   const int n = seq_lens[b], cap = max_pages * kPage;
   return n < 0 ? 0 : (n > cap ? cap : n);
 }
-__device__ __forceinline__ int pages_of(const int* seq_lens, int max_pages, int b) {
-  return (len_of(seq_lens, max_pages, b) + kPage - 1) / kPage;
+// Pages of sequence b in the split kernel's partition (0 for a short one).
+__device__ __forceinline__ int pages_of(const int* seq_lens, int max_pages, int q_len, int b) {
+  const int n = len_of(seq_lens, max_pages, b);
+  return is_short(n, q_len) ? 0 : (n + kPage - 1) / kPage;
 }
 // CTA that owns page x of the list when T pages are split over G CTAs.
 __device__ __forceinline__ int owner(long long x, long long T, int G) {
@@ -175,7 +176,7 @@ struct Segments {
     long long c = 0;
     for (int b0 = 0; b0 < p.B; b0 += 32) {
       const int bl = b0 + lane;
-      const long long w = bl < p.B ? (long long)p.Hkv * pages_of(p.seq_lens, p.max_pages, bl) : 0;
+      const long long w = bl < p.B ? (long long)p.Hkv * pages_of(p.seq_lens, p.max_pages, p.q_len, bl) : 0;
       long long inc = w;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -187,7 +188,7 @@ struct Segments {
         const int L = __ffs(hit) - 1;  // first sequence whose pages reach past lo
         const long long excl = c + __shfl_sync(0xffffffffu, inc - w, L);
         b = b0 + L;
-        P = pages_of(p.seq_lens, p.max_pages, b);
+        P = pages_of(p.seq_lens, p.max_pages, p.q_len, b);
         kvh = (int)((lo - excl) / P);
         pre = excl + (long long)kvh * P;
         return;
@@ -211,7 +212,7 @@ struct Segments {
       kvh = 0;
       do {
         ++b;
-        P = b < p.B ? pages_of(p.seq_lens, p.max_pages, b) : 1;
+        P = b < p.B ? pages_of(p.seq_lens, p.max_pages, p.q_len, b) : 1;
       } while (b < p.B && P == 0);
     }
   }
@@ -234,6 +235,15 @@ struct CombineParams {
   int q_len;       // query tokens per sequence
   int split_grid;  // CTAs launched for the split kernel
   int has_pool;    // 0: no page pool, every output is an empty attention
+  // rows of short sequences, computed here: queries, pools, table
+  const __nv_bfloat16* q;        // [B * Hq * q_len][D_qk]
+  const __nv_bfloat16* k_pages;  // [num_pages * 16][Hkv][D_qk]
+  const __nv_bfloat16* v_pages;  // [num_pages * 16][Hkv][D_v]
+  const int* block_table;
+  int num_pages;
+  float scale_log2;
+  int bounds_check;
+  int* status;
 };
 
 // One warp per (sequence, query head).  Before waiting for the split kernel
@@ -276,7 +286,81 @@ __device__ __forceinline__ void st_feats(__nv_bfloat16* dst, const uint32_t (&pk
   }
 }
 
-template <int DV>
+// Page id of token j of sequence b, or -1 if it lies outside the pool (such
+// a page reads as zeros, as the TMA copies of the split kernel read it).
+__device__ __forceinline__ int short_page(const CombineParams& p, int b, int j) {
+  const int pg = p.block_table[(size_t)b * p.max_pages + j / kPage];
+  if (pg < 0 || pg >= p.num_pages) {
+    if (p.bounds_check) atomicExch(p.status, kErrBounds);
+    return -1;
+  }
+  return pg;
+}
+
+// Row (b, h, token t) of a short sequence, by one warp in fp32, in one pass
+// over the visible cached tokens: lane l holds query features l*FQ ..
+// l*FQ+FQ-1 and value features l*FV .., each token's score is reduced across
+// the warp, and the online-softmax recurrence (running max, rescaled sum and
+// accumulator) runs on warp-uniform values.  Kept compact and out of line:
+// it serves rare rows, and its code in the kernel should cost nothing else.
+template <int DQK, int DV>
+__device__ __noinline__ void short_row(const CombineParams& p, int gw, int b, int h, int t, int lane) {
+  constexpr int FQ = DQK / 32, FV = DV / 32;
+  const int len = len_of(p.seq_lens, p.max_pages, b);
+  int vis = p.has_pool ? len - p.q_len + t + 1 : 0;  // tokens 0 .. vis - 1
+  vis = vis < 0 ? 0 : (vis > len ? len : vis);
+  const int kvh = h / p.group;
+  float qv[FQ];
+#pragma unroll
+  for (int f = 0; f < FQ; f += 2) {
+    const uint32_t w = *reinterpret_cast<const unsigned int*>(p.q + (size_t)gw * DQK + lane * FQ + f);
+    qv[f] = __uint_as_float(w << 16) * p.scale_log2;
+    qv[f + 1] = __uint_as_float(w & 0xFFFF0000u) * p.scale_log2;
+  }
+  float m = -INFINITY, l = 0.f, acc[FV];
+#pragma unroll
+  for (int f = 0; f < FV; ++f) acc[f] = 0.f;
+#pragma unroll 1
+  for (int j = 0; j < vis; ++j) {
+    const int pg = short_page(p, b, j);  // the same for every lane
+    const size_t tok = ((size_t)(pg < 0 ? 0 : pg) * kPage + j % kPage) * p.Hkv + kvh;
+    float s = 0.f;
+    if (pg >= 0) {
+#pragma unroll
+      for (int f = 0; f < FQ; f += 2) {
+        const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(p.k_pages + tok * DQK + lane * FQ + f));
+        s = fmaf(__uint_as_float(w << 16), qv[f], s);
+        s = fmaf(__uint_as_float(w & 0xFFFF0000u), qv[f + 1], s);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float m_new = fmaxf(m, s);
+    const float c = ex2_approx(m - m_new);  // 0 for the first token
+    const float e = ex2_approx(s - m_new);
+    m = m_new;
+    l = l * c + e;
+#pragma unroll
+    for (int f = 0; f < FV; f += 2) {
+      float v0 = 0.f, v1 = 0.f;
+      if (pg >= 0) {
+        const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(p.v_pages + tok * DV + lane * FV + f));
+        v0 = __uint_as_float(w << 16);
+        v1 = __uint_as_float(w & 0xFFFF0000u);
+      }
+      acc[f] = fmaf(e, v0, acc[f] * c);
+      acc[f + 1] = fmaf(e, v1, acc[f + 1] * c);
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  uint32_t pk[FV / 2];
+#pragma unroll
+  for (int f = 0; f < FV / 2; ++f) pk[f] = pack_bf16x2(acc[2 * f] * inv, acc[2 * f + 1] * inv);
+  st_feats<FV>(p.o + (size_t)gw * DV + lane * FV, pk);
+  if (lane == 0 && p.lse) p.lse[gw] = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
+}
+
+template <int DQK, int DV>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
   // The next decode's split kernel (a programmatic dependent) may launch and
   // set up while this grid runs; it waits for this grid before reading or
@@ -289,13 +373,21 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     return;
   }
   const int b = gw / (p.Hq * p.q_len), h = (gw / p.q_len) % p.Hq, kvh = h / p.group;
+  if (is_short(len_of(p.seq_lens, p.max_pages, b), p.q_len)) {
+    // Reads only the call's inputs, which the kernels before this call's
+    // split kernel had completed (that kernel waited for them before letting
+    // this grid launch): no wait needed before the row is computed.
+    short_row<DQK, DV>(p, gw, b, h, gw % p.q_len, lane);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }
   int nseg = 0;
   if (p.has_pool) {
     // pages of sequences before b, and in all (seq_lens is an input of the
     // split kernel, complete before it started)
     long long before = 0, T = 0;
     for (int bb = lane; bb < p.B; bb += 32) {
-      const long long w = pages_of(p.seq_lens, p.max_pages, bb);
+      const long long w = pages_of(p.seq_lens, p.max_pages, p.q_len, bb);
       T += w;
       if (bb < b) before += w;
     }
@@ -305,7 +397,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
       before += __shfl_xor_sync(0xffffffffu, before, o);
     }
     T *= p.Hkv;
-    const int P = pages_of(p.seq_lens, p.max_pages, b);
+    const int P = pages_of(p.seq_lens, p.max_pages, p.q_len, b);
     if (P > 0 && T > 0) {
       const long long G = split_ctas(T, p.split_grid);
       const long long pre = before * p.Hkv + (long long)kvh * P;
@@ -427,10 +519,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   auto pages_from_len = [&](int n) {
     const int cap = p.max_pages * kPage;
     n = n < 0 ? 0 : (n > cap ? cap : n);
-    return (n + kPage - 1) / kPage;
+    return is_short(n, p.q_len) ? 0 : (n + kPage - 1) / kPage;
   };
   long long T = (long long)pages_from_len(sl0) + pages_from_len(sl1);
-  for (int b = lane + 64; b < p.B; b += 32) T += pages_of(p.seq_lens, p.max_pages, b);
+  for (int b = lane + 64; b < p.B; b += 32) T += pages_of(p.seq_lens, p.max_pages, p.q_len, b);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
   T *= p.Hkv;
@@ -571,12 +663,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       };
       // O (+)= P V: P from TMEM over S (16 tokens = 8 columns per k-step), V
       // MN-major with its 64-feature boxes kBox apart.
-      // a_col = kFineCol: the residual of P in a fine segment.
-      auto issue_pv = [&](uint32_t gb, int nv, bool acc, uint32_t a_col) {
+      auto issue_pv = [&](uint32_t gb, int nv, bool acc) {
         const uint32_t stage = s_ring + (gb % nst) * C::STAGE;
         const uint64_t b0 = sw128_desc(stage + C::KB * kBox, kBox, 1024);
         for (int kk = 0; kk < nv; ++kk)
-          mma_f16_ts(tmem + kTmO, tS(gb) + a_col + kk * 8, b0 + ((kk * kPageBox) >> 4), C::IDESC_PV,
+          mma_f16_ts(tmem + kTmO, tS(gb) + kk * 8, b0 + ((kk * kPageBox) >> 4), C::IDESC_PV,
                      (acc || kk > 0) ? 1u : 0u);
       };
       while (seg.more() && ok) {
@@ -584,7 +675,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         long long pre;
         seg.take(b, kvh, pg_lo, pg_hi, pre, P);
         const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
-        const bool fine = seg_fine(P, p.q_len);
         const uint32_t qs = n_q % nqs;
         ok = mbar_wait(&sm.q_full[qs], (n_q / nqs) & 1, g);
         if (!ok) break;
@@ -621,8 +711,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (!ok) break;
           }
           tc_fence_after();
-          issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0, 0);
-          if (__builtin_expect(fine, 0)) issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), true, kFineCol);
+          issue_pv(gb, min(kBlkPages, pg_hi - (pg_lo + j * kBlkPages)), j > 0);
           tc_commit(&sm.kv_empty[gb % nst]);
           tc_commit(&sm.pv_done);
           if (has_next && !s_first) {
@@ -659,7 +748,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       seg.take(b, kvh, pg_lo, pg_hi, pre, P);
       const int len = len_of(p.seq_lens, p.max_pages, b);
       const int nb = (pg_hi - pg_lo + kBlkPages - 1) / kBlkPages;
-      const bool fine = seg_fine(P, p.q_len);
       // l_run: exact fp32 row sum (gives the LSE); l_rnd: sum of the rounded P
       // the MMA multiplies (normalises o so its weights sum to one).
       float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
@@ -733,44 +821,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           pk[q2] = bb;
           rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(bb << 16), __uint_as_float(bb & 0xFFFF0000u)));
         }
-        if (__builtin_expect(!fine, 1)) {
-          tmem_st32(tS, pk);
-        } else {
-          // The two-part product: S is still in TMEM (P has not gone over it
-          // yet); P is recomputed exactly as above, rounded (as pk) and its
-          // rounding residual stored to columns kFineCol on.  Kept out of the
-          // loop above, whose registers and schedule it would otherwise change.
-          tmem_ld64(tS, sr);
-          if (seen < kBlkTok) {
-#pragma unroll
-            for (int i = 0; i < kBlkTok; ++i)
-              if (i >= seen) sr[i] = 0xFF800000u;  // -inf
-          }
-#pragma unroll
-          for (int c8 = 0; c8 < kBlkTok / 16; ++c8) {  // 8 pairs (TMEM columns) at a time
-            uint32_t hi8[8], lo8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int q2 = c8 * 8 + i;
-              const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * q2]), __uint_as_float(sr[2 * q2 + 1])), sc2, nm2);
-              float p0, p1;
-              if ((q2 & 7) >= 6) {
-                f2_split(exp2_poly2(x2), p0, p1);
-              } else {
-                float x0, x1;
-                f2_split(x2, x0, x1);
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
-              hi8[i] = pack_bf16x2(p0, p1);
-              const float h0 = __uint_as_float(hi8[i] << 16), h1 = __uint_as_float(hi8[i] & 0xFFFF0000u);
-              lo8[i] = pack_bf16x2(p0 - h0, p1 - h1);  // P - h is exact in fp32
-              rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(lo8[i] << 16), __uint_as_float(lo8[i] & 0xFFFF0000u)));
-            }
-            tmem_st8(tS + c8 * 8, hi8);
-            tmem_st8(tS + kFineCol + c8 * 8, lo8);
-          }
-        }
         {
           const uint64_t a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
           const uint64_t bq = add2(add2(rr2[0], rr2[1]), add2(rr2[2], rr2[3]));
@@ -780,6 +830,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           l_run += a0 + a1;
           l_rnd += b0 + b1;
         }
+        tmem_st32(tS, pk);
         if (warp == 0 && valid < nv * kPage) {
           // Tokens past the end of the sequence inside its last page: P is 0
           // there, but the cache slots may hold anything (0 * NaN = NaN), so
@@ -978,6 +1029,14 @@ int run_decode(const DecodeArgs& a, cudaStream_t stream) {
   // Without a pool the split kernel did not run: the combine then treats
   // every sequence as empty (O = 0, LSE = -inf).
   cp.has_pool = has_pool ? 1 : 0;
+  cp.q = static_cast<const __nv_bfloat16*>(a.q);
+  cp.k_pages = static_cast<const __nv_bfloat16*>(a.k_pages);
+  cp.v_pages = static_cast<const __nv_bfloat16*>(a.v_pages);
+  cp.block_table = a.block_table;
+  cp.num_pages = a.num_pages;
+  cp.scale_log2 = a.scale * kLog2e;
+  cp.bounds_check = (debug_flags() & 1) ? 1 : 0;
+  cp.status = status;
   const int nw = a.B * a.Hq * q_len;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((nw + 7) / 8);
@@ -989,7 +1048,7 @@ int run_decode(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<DV>, cp);
+  err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<DQK, DV>, cp);
   if (err == cudaSuccess) err = cudaGetLastError();
   return err == cudaSuccess ? 0 : fail_cuda("decode: combine launch", err);
 }
