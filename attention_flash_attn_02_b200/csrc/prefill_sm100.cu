@@ -853,8 +853,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               p_pairs_fine<FP8, kRsum, E5M2, Q_LO, Q_HI>(sr, sc2, nm2, rs2, rr2, pk, pk_lo, tS);
             } else {
               // (the exponent polynomial only in the kernels for plain tiles)
-              p_pairs<FP8, kRsum, false, Q_LO, Q_HI, false, FINE ? 0 : kEmuPairsPer8<FP8>>(sr, sc2, nm2, rs2, rr2,
-                                                                                           pk, pk_lo);
+              // (plain tiles normalise by the exact sum: no rounded sum here)
+              p_pairs<FP8, ATTN_ROUNDED_SUM != 0, false, Q_LO, Q_HI, false, FINE ? 0 : kEmuPairsPer8<FP8>>(
+                  sr, sc2, nm2, rs2, rr2, pk, pk_lo);
               tmem_st_cols<C0, C1>(tS, pk);
             }
           };
