@@ -14,30 +14,38 @@
 //   bwd_kernel        one CTA per 128-key K/V tile of one K/V head, looping
 //                     over the query heads of its group and the 128-row
 //                     query blocks that see the tile.  Per CTA:
-//       warp 8       TMA producer: K_j and V_j once, then Q_i and dO_i
-//                    (double buffered) per step.
+//       warp 8       TMA producer and reducer, one thread: K_j and V_j
+//                    once; per step the Q_i and dO_i tiles (double
+//                    buffered), each loaded into its buffer right after that
+//                    buffer's dQ staging from two steps back has been added
+//                    to the fp32 dQ accumulator by a bulk tensor reduction
+//                    (the loads then do not queue behind other reductions).
 //       warp 9       TMEM owner; one thread issues per step
 //                      dP^T = V_j dO_i^T                        (TMEM),
 //                    then, once P^T and dS^T are written back,
-//                      dV += P^T dO_i   and  dK += dS^T Q_i      (A from TMEM)
+//                      dV += P^T dO_i                           (A from TMEM)
+//                      S^T = K_j Q_{i'}^T of the next step (if Q_{i'} is in)
+//                      dK += dS^T Q_i                           (A from TMEM)
 //                      dQ_i = dS K_j                            (A from smem)
-//                    and S^T = K_j Q_{i'}^T of the next step, which runs
-//                    while dQ_i is read out.
-//       warps 0-3    one thread per key (TMEM lane): P^T of its key against
-//                    the block's 128 queries as soon as S^T is there (back to
-//                    TMEM as bf16), then dS^T once dP^T is (back to TMEM, and
-//                    dS (bf16) into a swizzled shared-memory tile).
-//       warps 4-7    one thread per query row: dQ_i from TMEM into a
-//                    128-byte-swizzled fp32 staging tile (the dS tile, free
-//                    between the dQ product and the next step's dS), which
-//                    the TMA unit adds to the fp32 accumulator with bulk
-//                    tensor reductions, 64 features at a time.
-//                    At the end warps 0-3 write dK (times scale) and dV.
+//                    so that the next P^T is formed while dK and dQ_i run.
+//       warps 0-7    two warps per TMEM lane quadrant, each over 64 of the
+//                    block's 128 queries: P^T of the warp's keys (one thread
+//                    per key = TMEM lane) as soon as S^T is there, back to
+//                    TMEM as bf16; the previous step's dQ_i, whenever it is
+//                    complete, from TMEM (one thread per query row, half of
+//                    the features each) into 128-byte-swizzled fp32 staging
+//                    boxes in that step's Q buffer (first half of the
+//                    features) and dO buffer (second half), which no product
+//                    reads once dQ_i is done; then dS^T once dP^T is there,
+//                    back to TMEM, and dS (bf16) into a swizzled shared-memory
+//                    tile.  At the end each writes its half of dK (times
+//                    scale) and dV.
 //   bwd_post_kernel   dQ = bf16(scale * accumulator).
-// TMEM (512 columns): [0,128) S^T, then P^T over its first 64; [128,256)
-// dP^T, then dS^T over its first 64, then dQ_i; [256,384) dV; [384,512) dK.
-// So the next step's S^T can be computed, and its P^T formed, while dQ_i is
-// still being read out; only dP^T waits for the read-out.
+// TMEM (512 columns): [0,128) S^T, then P^T packed over columns 0-31 (queries
+// 0-63) and 64-95 (queries 64-127); [128,256) dP^T, then dS^T packed the same
+// way, then dQ_i; [256,384) dV; [384,512) dK.  So the next step's S^T can be
+// computed, and its P^T formed, while dK and dQ_i run and dQ_i is read out;
+// only dP^T waits for the read-out.
 // Every operand tile is a 128-row, 128-byte-swizzled TMA tile, used K-major
 // or MN-major by its descriptor; dS is stored [key][query] so that dQ reads
 // it MN-major.
@@ -94,11 +102,10 @@ struct BParams {
 };
 
 struct BSmem {
-  uint64_t kv_full, q_full[2], q_empty[2];
-  uint64_t s_full, dp_full, p_full, dq_full, dq_empty, ds_empty, fin, drain;
-  uint64_t stat;  // a step's LSE/Dvec written to shared memory (128 arrivals)
-  uint64_t stg_full;  // dQ staging written (128 arrivals, per 64-feature half)
-  uint64_t stg_free;  // ... and read by the bulk reduction (1 arrival)
+  uint64_t kv_full, q_full[2], do_full[2];
+  uint64_t s_full, dp_full, p_full, dq_full, dq_empty, fin, drain;
+  uint64_t stat[2];  // [step & 1]: the step's LSE/Dvec written to shared memory (128 arrivals)
+  uint64_t stg_q[2], stg_do[2];  // [step & 1]: a half of the step's dQ staged (128 arrivals each)
   uint32_t tmem_base;
   int abort_flag;
   float lse2[2][kT];  // [buffer][query]
@@ -120,8 +127,10 @@ __device__ __forceinline__ void query_range(const BParams& p, int k0, int k1, in
   r_hi = r_hi > p.Lq ? p.Lq : r_hi;
 }
 
-// The dQ staging (two fp32 boxes of 128 rows x 32 features) reuses the dS tile.
-static_assert(2 * BCfg<128>::BOX_BYTES == BCfg<128>::DS_BYTES, "dQ staging fills the dS tile");
+// The dQ staging (D/32 fp32 boxes of 128 rows x 32 features) fills the step's
+// dO and Q buffers exactly.
+static_assert(BCfg<128>::TILE_BYTES == 2 * BCfg<128>::BOX_BYTES && BCfg<64>::TILE_BYTES == BCfg<64>::BOX_BYTES,
+              "dQ staging fills the step's dO and Q buffers");
 
 template <int D>
 constexpr bool bwd_fits() {
@@ -135,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dq, const BParams p) {
   using C = BCfg<D>;
-  constexpr int kDqHalves = D / 64;  // dQ leaves TMEM 64 features (two fp32 boxes) at a time
+  constexpr int kDqBoxes = D / 32;  // fp32 boxes of 32 features per dQ block
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   if ((base & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned base
@@ -161,19 +170,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.kv_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.q_full[s], 1);
-      mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.do_full[s], 1);
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.dp_full, 1);
-    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.p_full, 256);
     mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, 128);
-    mbar_init(&sm.ds_empty, 1);
+    mbar_init(&sm.dq_empty, 256);
     mbar_init(&sm.fin, 1);
     mbar_init(&sm.drain, 1);
-    mbar_init(&sm.stat, 128);
-    mbar_init(&sm.stg_full, 128);
-    mbar_init(&sm.stg_free, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sm.stat[t], 128);
+      mbar_init(&sm.stg_q[t], 128);
+      mbar_init(&sm.stg_do[t], 128);
+    }
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -208,22 +218,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(base + C::OFF_K + bx * C::BOX_BYTES, &tm_k, &sm.kv_full, bx * 64, k0, bkv);
         tma_load_3d(base + C::OFF_V + bx * C::BOX_BYTES, &tm_v, &sm.kv_full, bx * 64, k0, bkv);
       }
+      // Step t's dQ staging, a half at a time, into the fp32 accumulator
+      // with bulk tensor reductions (rows past Lq fall outside the tensor map
+      // and are not written); each half's buffer is reloaded right after it
+      // has been read, so the loads do not queue behind the other half.
+      auto reduce_half = [&](int t, int h) {
+        const int ts = t & 1;
+        if (!mbar_wait(h == 0 ? &sm.stg_q[ts] : &sm.stg_do[ts], (t >> 1) & 1, g)) return false;
+        const int bh = b * p.Hq + step_head(t), r0 = step_blk(t) * kT;
+        const uint32_t src = base + (h == 0 ? C::OFF_Q : C::OFF_DO) + ts * C::TILE_BYTES;
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_reduce_add_3d(&tm_dq, src + bx * C::BOX_BYTES, h * (D / 2) + bx * 32, r0, bh);
+        bulk_commit_group();
+        bulk_wait_read<0>();
+        return true;
+      };
       for (int s = 0; s < nsteps && ok; ++s) {
         const int qs = s & 1;
-        if (s >= 2) ok = mbar_wait(&sm.q_empty[qs], ((s >> 1) - 1) & 1, g);
-        if (!ok) break;
         const int bh = b * p.Hq + step_head(s), r0 = step_blk(s) * kT;
-        mbar_arrive_expect_tx(&sm.q_full[qs], 2 * C::TILE_BYTES);
-        for (int bx = 0; bx < C::NBOX; ++bx) {
+        if (s >= 2) ok = reduce_half(s - 2, 0);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&sm.q_full[qs], C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_3d(base + C::OFF_Q + qs * C::TILE_BYTES + bx * C::BOX_BYTES, &tm_q, &sm.q_full[qs], bx * 64,
                       r0, bh);
-          tma_load_3d(base + C::OFF_DO + qs * C::TILE_BYTES + bx * C::BOX_BYTES, &tm_do, &sm.q_full[qs],
+        if (s >= 2) ok = reduce_half(s - 2, 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&sm.do_full[qs], C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_3d(base + C::OFF_DO + qs * C::TILE_BYTES + bx * C::BOX_BYTES, &tm_do, &sm.do_full[qs],
                       bx * 64, r0, bh);
-        }
       }
+      for (int t = (nsteps > 2 ? nsteps - 2 : 0); t < nsteps && ok; ++t) ok = reduce_half(t, 0) && reduce_half(t, 1);
+      bulk_wait_all();  // every reduction has completed
       // Drain: the last loads have landed before the CTA exits.
       mbar_wait(&sm.kv_full, 0, g_drain);
-      for (int s = (nsteps > 2 ? nsteps - 2 : 0); s < nsteps; ++s) mbar_wait(&sm.q_full[s & 1], (s >> 1) & 1, g_drain);
+      for (int s = (nsteps > 2 ? nsteps - 2 : 0); s < nsteps; ++s) {
+        mbar_wait(&sm.q_full[s & 1], (s >> 1) & 1, g_drain);
+        mbar_wait(&sm.do_full[s & 1], (s >> 1) & 1, g_drain);
+      }
     }
     finish();
   } else if (warp == 9) {
@@ -235,6 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dv_desc = sw128_desc(base + C::OFF_V, 16, 1024);   // V_j K-major (dP^T A)
       const uint64_t kmn_desc = sw128_desc(base + C::OFF_K, C::BOX_BYTES, 1024);  // K_j MN-major (dQ B)
       const uint64_t ds_desc = sw128_desc(base + C::OFF_DS, C::BOX_BYTES, 1024);  // dS MN-major (dQ A)
+      // packed bf16 P^T / dS^T column of k-step kk (16 queries): queries 0-63
+      // at columns 0-31 of their region, queries 64-127 at columns 64-95
+      auto a_col = [](int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); };
       // S^T = K_j Q_i^T of step s into TM_S, k-steps of 16 features
       auto issue_st = [&](int s) {
         const uint64_t q_km = sw128_desc(base + C::OFF_Q + (s & 1) * C::TILE_BYTES, 16, 1024);
@@ -261,6 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t q_tile = base + C::OFF_Q + qs * C::TILE_BYTES;
         const uint32_t do_tile = base + C::OFF_DO + qs * C::TILE_BYTES;
         const uint64_t do_km = sw128_desc(do_tile, 16, 1024);
+        ok = mbar_wait(&sm.do_full[qs], (s >> 1) & 1, g);
+        if (!ok) break;
+        tc_fence_after();
         // dP^T = V_j dO_i^T
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -272,30 +312,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(&sm.p_full, s & 1, g);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dO_i, dK += dS^T Q_i (A from TMEM, 16 queries = 8 columns
-        // per k-step; B MN-major, 16 rows = 2 KB per k-step)
+        // dV += P^T dO_i (A from TMEM, 16 queries = 8 columns per k-step; B
+        // MN-major, 16 rows = 2 KB per k-step)
         const uint64_t do_mn = sw128_desc(do_tile, C::BOX_BYTES, 1024);
         const uint64_t q_mn = sw128_desc(q_tile, C::BOX_BYTES, 1024);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk) {
           const uint32_t off = (kk * 16 * 128) >> 4;
-          mma_f16_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, do_mn + off, C::ID_ACC, (s > 0 || kk > 0) ? 1u : 0u);
-          mma_f16_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, q_mn + off, C::ID_ACC, (s > 0 || kk > 0) ? 1u : 0u);
+          mma_f16_ts(tmem + C::TM_DV, tmem + C::TM_S + a_col(kk), do_mn + off, C::ID_ACC, (s > 0 || kk > 0) ? 1u : 0u);
+        }
+        // The next step's S^T, before dK and dQ when its Q block is in, so
+        // that its P^T is formed while they run (its columns' last reader,
+        // dV, was issued above, and MMAs run in issue order); else after them.
+        const bool st_next = s + 1 < nsteps;
+        const uint32_t q_par = ((s + 1) >> 1) & 1;
+        bool st_early = st_next && mbar_test(&sm.q_full[(s + 1) & 1], q_par);
+        if (st_early) {
+          tc_fence_after();
+          issue_st(s + 1);
+        }
+        // dK += dS^T Q_i (A from TMEM)
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk) {
+          const uint32_t off = (kk * 16 * 128) >> 4;
+          mma_f16_ts(tmem + C::TM_DK, tmem + C::TM_DP + a_col(kk), q_mn + off, C::ID_ACC, (s > 0 || kk > 0) ? 1u : 0u);
         }
         // dQ_i = dS K_j over the tile's 128 keys (both operands MN-major),
-        // into the dP^T columns: issued after dK, their last reader
+        // into the dP^T columns: issued after dK, their last reader.  Its
+        // completion also frees the step's Q and dO buffers (dQ staging).
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk) {
           const uint32_t off = (kk * 16 * 128) >> 4;
           mma_f16_ss(tmem + C::TM_DP, ds_desc + off, kmn_desc + off, C::ID_DQ, kk > 0);
         }
         tc_commit(&sm.dq_full);
-        tc_commit(&sm.q_empty[qs]);
-        tc_commit(&sm.ds_empty);
-        // The next step's S^T: its columns' last reader (dV, P^T) was issued
-        // above, and MMAs run in issue order.
-        if (s + 1 < nsteps) {
-          ok = mbar_wait(&sm.q_full[(s + 1) & 1], ((s + 1) >> 1) & 1, g);
+        if (st_next && !st_early) {
+          ok = mbar_wait(&sm.q_full[(s + 1) & 1], q_par, g);
           if (!ok) break;
           tc_fence_after();
           issue_st(s + 1);
@@ -307,35 +359,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     finish();
-  } else if (warp < 4) {
-    // ------------------------------------------------- per-key P^T and dS^T
-    const int r = warp * 32 + lane;  // key row of the tile = TMEM lane
+  } else if (warp < 8) {
+    // -------------------- P^T, dS^T and the dQ_i read-out: two warps per TMEM
+    // lane quadrant, each over 64 of the block's 128 queries (or of dQ_i's
+    // features)
+    const int quad = warp & 3, hf = warp >> 2;
+    const int r = quad * 32 + lane;  // TMEM lane: key row (P^T, dS^T), query row (dQ_i)
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const int q0 = hf * 64;  // this warp's queries of the block
+    // its S^T and dP^T columns; packed bf16 P^T and dS^T go over the first 32
+    const uint32_t c_s = tmem + C::TM_S + hf * 64 + lane_off, c_dp = tmem + C::TM_DP + hf * 64 + lane_off;
     const int key = k0 + r;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int off = p.Lk - p.Lq;
     bool ok = true;
-    // LSE (log2) and Dvec of query r of step s's block; each thread loads one
-    // of the 128 and shares it through shared memory.
+    // LSE (log2) and Dvec of query r of step s's block; the threads of the
+    // first four warps each load one of the 128 and share it through shared
+    // memory.  Step s's values are in place once `stat[s & 1]` completes its
+    // phase s / 2 (an mbarrier, so the wait is bounded); step s + 2's go into
+    // the same buffer once step s + 1's dP^T is complete, which is after every
+    // thread is done with step s (dP^T is issued after all of step s's dS^T).
     auto load_stat = [&](int s, float& l2v, float& dvv) {
       const int q = step_blk(s) * kT + r;
       const size_t row = (size_t)(b * p.Hq + step_head(s)) * p.Lq + q;
       l2v = q < p.Lq ? p.lse2[row] : INFINITY;
       dvv = q < p.Lq ? p.dvec[row] : 0.f;
     };
-    // All 128 values of step s are in place once every thread has arrived on
-    // `stat` (an mbarrier, so the wait is bounded).  Step s + 1's values go
-    // into the other buffer once step s's softmax is done, which is also
-    // after every thread is done with step s - 1, the buffer's last user.
     auto put_stat = [&](int s, float l2v, float dvv) {
       sm.lse2[s & 1][r] = l2v;
       sm.dvec[s & 1][r] = dvv;
-      mbar_arrive(&sm.stat);
+      mbar_arrive(&sm.stat[s & 1]);
     };
-    if (nsteps > 0) {
+    if (nsteps > 0 && hf == 0) {
       float l2v, dvv;
       load_stat(0, l2v, dvv);
       put_stat(0, l2v, dvv);
     }
+    // dQ_i of step t: this warp's D/2 features of its query row out of TMEM
+    // (the columns then take the next dP^T), then into its half's staging
+    // boxes (32 features each) in step t's Q buffer (first half) or dO buffer
+    // (second half), which no product reads any more (dQ_i was the step's
+    // last): row r's 8 chunks of 16 bytes, XOR-swizzled by the row's low 3
+    // bits (the 128-byte swizzle of the reduction's tensor map).
+    auto dq_out = [&](int t) {
+      tc_fence_after();
+      uint32_t v[D / 2];
+      if constexpr (D == 128) {
+        tmem_ld64(tmem + C::TM_DP + lane_off + hf * 64, v);
+      } else {
+        tmem_ld32(tmem + C::TM_DP + lane_off + hf * 32, v);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.dq_empty);
+      const uint32_t stage = base + (hf == 0 ? C::OFF_Q : C::OFF_DO) + (t & 1) * C::TILE_BYTES;
+#pragma unroll
+      for (int bx = 0; bx < D / 64; ++bx)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t a = stage + bx * C::BOX_BYTES + r * 128 + ((u ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[bx * 32 + 4 * u]),
+                       "r"(v[bx * 32 + 4 * u + 1]), "r"(v[bx * 32 + 4 * u + 2]), "r"(v[bx * 32 + 4 * u + 3])
+                       : "memory");
+        }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging visible to the TMA unit
+      mbar_arrive(hf == 0 ? &sm.stg_q[t & 1] : &sm.stg_do[t & 1]);
+    };
     // visible queries of this key: q + off >= key (causal), q + off - W + 1 <= key (window)
     const int q_first = p.causal ? key - off : INT_MIN;
     const int q_last = (p.causal && p.window > 0) ? key - off + p.window - 1 : INT_MAX;
@@ -344,31 +431,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = step_blk(s);
       const int buf = s & 1;
       float nl2 = INFINITY, ndv = 0.f;  // the next step's values, loaded early
-      if (s + 1 < nsteps) load_stat(s + 1, nl2, ndv);
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.stat, s & 1, g));
-      if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full, s & 1, g));
+      if (hf == 0 && s + 1 < nsteps) load_stat(s + 1, nl2, ndv);
+      // Wait for S^T, reading the previous step's dQ out meanwhile if it
+      // completes first (a bounded wait, like mbar_wait's).
+      bool dq_pending = s > 0;
+      {
+        bool got = false;
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 0; it < (1u << 28); ++it) {
+          if (dq_pending && __all_sync(0xffffffffu, mbar_test(&sm.dq_full, (s - 1) & 1))) {
+            dq_out(s - 1);
+            dq_pending = false;
+          }
+          got = __all_sync(0xffffffffu, mbar_test(&sm.s_full, s & 1));
+          if (got || ((it & 31u) == 31u && __any_sync(0xffffffffu, *g.abort_flag != 0 ||
+                                                                        globaltimer_ns() - t0 > g.timeout_ns)))
+            break;
+        }
+        if (!got) {
+          if (lane == 0 && !*g.abort_flag) {
+            *g.abort_flag = 1;
+            atomicExch(p.status, kErrTimeout);
+          }
+          ok = false;
+          break;
+        }
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.stat[buf], (s >> 1) & 1, g));
       if (!ok) break;
       tc_fence_after();
-      // P^T from S^T (masked entries 0), back to TMEM as bf16 over S^T's
-      // first 64 columns; the packed values stay for dS.
-      uint32_t pp[kT / 2];
-      // a key that sees every query of the block needs no per-element test
-      // (rows past Lq have LSE +inf, so their P is 0 either way)
-      const bool all_vis = __all_sync(0xffffffffu, key_ok && i * kT >= q_first && i * kT + kT - 1 <= q_last);
+      // P^T from S^T (masked entries 0), back to TMEM as bf16.  A key that
+      // sees all of the warp's queries needs no per-element test (rows past
+      // Lq have LSE +inf, so their P is 0 either way).
+      const int qb = i * kT + q0;
+      const bool all_vis = __all_sync(0xffffffffu, key_ok && qb >= q_first && qb + 63 <= q_last);
+      uint32_t sr[64];  // this warp's 64 S^T columns, loaded together
+      tmem_ld32_async(c_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32_async(c_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      tmem_ld_wait(sr);
 #pragma unroll
-      for (int c = 0; c < kT / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tmem + C::TM_S + lane_off + c * 32, sr);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pp[16];
+        const float* l2 = &sm.lse2[buf][q0 + c * 32];
         if (all_vis) {
 #pragma unroll
           for (int t = 0; t < 32; t += 2) {
-            const uint64_t x2 = fma2(f2(__uint_as_float(sr[t]), __uint_as_float(sr[t + 1])),
-                                     f2(p.scale_log2, p.scale_log2),
-                                     f2(-sm.lse2[buf][c * 32 + t], -sm.lse2[buf][c * 32 + t + 1]));
+            const uint64_t x2 = fma2(f2(__uint_as_float(sr[c * 32 + t]), __uint_as_float(sr[c * 32 + t + 1])),
+                                     f2(p.scale_log2, p.scale_log2), f2(-l2[t], -l2[t + 1]));
             float x0, x1;
             f2_split(x2, x0, x1);
-            pp[c * 16 + t / 2] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+            pp[t / 2] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
           }
         } else {
 #pragma unroll
@@ -376,46 +488,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             float pv[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int qq = c * 32 + t + e;
-              const int q = i * kT + qq;
+              const int q = qb + c * 32 + t + e;
               const bool vis = key_ok && q >= q_first && q <= q_last;
-              const float x = fmaf(__uint_as_float(sr[t + e]), p.scale_log2, -sm.lse2[buf][qq]);
+              const float x = fmaf(__uint_as_float(sr[c * 32 + t + e]), p.scale_log2, -l2[t + e]);
               pv[e] = vis ? ex2_approx(x) : 0.f;
             }
-            pp[c * 16 + t / 2] = pack_bf16x2(pv[0], pv[1]);
+            pp[t / 2] = pack_bf16x2(pv[0], pv[1]);
           }
         }
-        tmem_st16(tmem + C::TM_S + lane_off + c * 16, pp + c * 16);
+        tmem_st16(c_s + c * 16, pp);
       }
+      tmem_st_wait();  // P^T is read back below
+      if (dq_pending) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (s - 1) & 1, g));
+        if (!ok) break;
+        dq_out(s - 1);
+      }
+      // dP^T complete also means the previous dQ product, the dS tile's last
+      // reader, is (it was issued before dP^T)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.dp_full, s & 1, g));
       if (!ok) break;
-      if (s > 0) {  // the dS tile is free once the previous dQ has left its staging
-        const uint32_t n_last = (uint32_t)s * kDqHalves - 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.stg_free, n_last & 1, g));
-        if (!ok) break;
-      }
       tc_fence_after();
       // dS = P (dP - Dvec), with P as rounded for the dV product
+      uint32_t dr[64], pw[32];  // dP^T and the packed P^T of this warp's queries, loaded together
+      tmem_ld32_async(c_dp, *reinterpret_cast<uint32_t(*)[32]>(dr));
+      tmem_ld32_async(c_dp + 32, *reinterpret_cast<uint32_t(*)[32]>(dr + 32));
+      tmem_ld32_async(c_s, pw);
+      tmem_ld_wait(dr, pw);
 #pragma unroll
-      for (int c = 0; c < kT / 32; ++c) {
-        uint32_t dr[32];
-        tmem_ld32(tmem + C::TM_DP + lane_off + c * 32, dr);
+      for (int c = 0; c < 2; ++c) {
         uint32_t dd[16];
+        const float* dv = &sm.dvec[buf][q0 + c * 32];
 #pragma unroll
         for (int t = 0; t < 32; t += 2) {
-          const uint32_t pw = pp[c * 16 + t / 2];
-          const float p0 = __uint_as_float(pw << 16), p1 = __uint_as_float(pw & 0xFFFF0000u);
-          const int qq = c * 32 + t;
-          dd[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dr[t]) - sm.dvec[buf][qq]),
-                                  p1 * (__uint_as_float(dr[t + 1]) - sm.dvec[buf][qq + 1]));
+          const uint32_t w = pw[c * 16 + t / 2];
+          const float p0 = __uint_as_float(w << 16), p1 = __uint_as_float(w & 0xFFFF0000u);
+          dd[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dr[c * 32 + t]) - dv[t]),
+                                  p1 * (__uint_as_float(dr[c * 32 + t + 1]) - dv[t + 1]));
         }
-        tmem_st16(tmem + C::TM_DP + lane_off + c * 16, dd);
-        // dS row (queries c*32 .. c*32+31 of key r) into the swizzled tile:
+        tmem_st16(c_dp + c * 16, dd);
+        // dS row (queries q0 + c*32 .. +31 of key r) into the swizzled tile:
         // 64-query boxes, 16-byte chunks XORed with the row's low 3 bits
-        const int bx = (c * 32) / 64, ch0 = ((c * 32) % 64) / 8;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t a = base + C::OFF_DS + bx * C::BOX_BYTES + r * 128 + (((ch0 + u) ^ (r & 7)) << 4);
+          const uint32_t a = base + C::OFF_DS + hf * C::BOX_BYTES + r * 128 + (((c * 4 + u) ^ (r & 7)) << 4);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(dd[4 * u]), "r"(dd[4 * u + 1]),
                        "r"(dd[4 * u + 2]), "r"(dd[4 * u + 3])
                        : "memory");
@@ -425,15 +541,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // dS visible to the tensor core
       tc_fence_before();
       mbar_arrive(&sm.p_full);
-      if (s + 1 < nsteps) put_stat(s + 1, nl2, ndv);
+      if (hf == 0 && s + 1 < nsteps) put_stat(s + 1, nl2, ndv);
     }
-    // dK (times scale) and dV of this key row
+    if (ok && nsteps > 0) {  // the last step's dQ
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (nsteps - 1) & 1, g));
+      if (ok) dq_out(nsteps - 1);
+    }
+    // dK (times scale) and dV of this key row, this warp's D/2 features
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.fin, 0, g));
     if (ok) {
       tc_fence_after();
       const size_t row = (size_t)bkv * p.Lk + key;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {
         uint32_t kr[32], vr[32];
         if (nsteps > 0) {
           tmem_ld32(tmem + C::TM_DK + lane_off + c * 32, kr);
@@ -460,64 +580,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    finish();
-  } else if (warp < 8) {
-    // ------------------------------------------------ dQ_i into the accumulator
-    const int r = (warp & 3) * 32 + lane;  // query row of the block = TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const bool leader = threadIdx.x == 4 * 32;  // issues the bulk reductions
-    const uint32_t stage = base + C::OFF_DS;    // two 32-feature fp32 boxes of BOX_BYTES (16 KB)
-    uint32_t n_use = 0;                         // staging uses so far
-    bool ok = true;
-    for (int s = 0; s < nsteps && ok; ++s) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, s & 1, g));
-      if (!ok) break;
-      tc_fence_after();
-      const int bh = b * p.Hq + step_head(s), r0 = step_blk(s) * kT;
-      // All of dQ_i out of TMEM first (its columns then take the next dP^T),
-      // then through the staging tile 64 features at a time.
-      uint32_t v[kDqHalves][64];
-#pragma unroll
-      for (int h = 0; h < kDqHalves; ++h) {
-        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v[h]));
-        tmem_ld32(tmem + C::TM_DP + lane_off + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v[h] + 32));
-      }
-      tc_fence_before();
-      mbar_arrive(&sm.dq_empty);
-#pragma unroll
-      for (int h = 0; h < kDqHalves; ++h, ++n_use) {
-        if (n_use > 0) {  // the staging tile's previous contents have been read
-          ok = __all_sync(0xffffffffu, mbar_wait(&sm.stg_free, (n_use - 1) & 1, g));
-          if (!ok) break;
-        }
-        // row r of both boxes: 8 chunks of 16 bytes each, XOR-swizzled by the
-        // row's low 3 bits (the 128-byte swizzle of the reduction's tensor map)
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t a = stage + bb * C::BOX_BYTES + r * 128 + ((u ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[h][bb * 32 + 4 * u]),
-                         "r"(v[h][bb * 32 + 4 * u + 1]), "r"(v[h][bb * 32 + 4 * u + 2]), "r"(v[h][bb * 32 + 4 * u + 3])
-                         : "memory");
-          }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging visible to the TMA unit
-        mbar_arrive(&sm.stg_full);
-        if (leader) {
-          ok = mbar_wait(&sm.stg_full, n_use & 1, g);
-          if (ok) {
-            // rows past Lq fall outside the tensor map and are not written
-            tma_reduce_add_3d(&tm_dq, stage, h * 64, r0, bh);
-            tma_reduce_add_3d(&tm_dq, stage + C::BOX_BYTES, h * 64 + 32, r0, bh);
-            bulk_commit_group();
-            bulk_wait_read_all();
-            mbar_arrive(&sm.stg_free);
-          }
-        }
-        ok = __all_sync(0xffffffffu, ok);
-      }
-    }
-    if (leader) bulk_wait_all();  // every reduction has completed
     finish();
   } else {
     finish();  // warps 10-11

@@ -96,6 +96,7 @@ PROFILE_WORKLOADS = {
     "e5m2": (dataclasses.replace(FP8_CAUSAL, name="fp8_causal_B1_H32_L16384_D128", Lq=16384, Lk=16384), 4, "e5m2"),
     "latent256": (LATENT_256, 3, "mla"),
     "decode": (MQA_DECODE, 2, "decode"),
+    "backward": (GQA_CAUSAL, 1, "bwd"),
 }
 
 
@@ -117,6 +118,13 @@ def run_profile(args):
         q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
         call = attn.attn_fwd_fp8 if kind == "e4m3" else attn.attn_fwd_e5m2
         fn = lambda: call(q8, k8, v8, sq, sk, sv, shape.scale, shape.causal, shape.window)  # noqa: E731
+    elif kind == "bwd":
+        # one forward for O and LSE, then the backward launches alone
+        q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(idx))]
+        g = torch.Generator().manual_seed(seed_of(idx) + 300)
+        do = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+        o, lse = attn.attn_fwd(q, k, v, shape.scale, shape.causal, shape.window)
+        fn = lambda: attn.attn_bwd(q, k, v, o, do, lse, shape.scale, shape.causal, shape.window)  # noqa: E731
     else:
         q, k, v = [t.to(dev) for t in prefill_inputs(shape, seed_of(idx))]
         call = attn.attn_fwd_mla if kind == "mla" else attn.attn_fwd
