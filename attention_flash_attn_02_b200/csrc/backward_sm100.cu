@@ -144,7 +144,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dq, const BParams p) {
   using C = BCfg<D>;
-  constexpr int kDqBoxes = D / 32;  // fp32 boxes of 32 features per dQ block
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   if ((base & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned base
