@@ -985,25 +985,27 @@ int launch_range(const PrefillArgs& a, Params p, int mg_lo, int mg_hi, const CUt
   }
   p.mg_hi = mg_hi;
   p.n_units = p.n_pairs * (mg_hi - mg_lo);
+  // The loads carry L2 policies (Q evict-first, K/V evict-last) and O goes
+  // out with streaming stores: K/V stay in L2 for the other units that read
+  // them.  On the GQA causal workload that cut the reads from 308 to 245 MB
+  // per launch (traffic 1.24x -> 1.01x of the algorithmic bytes) at the same
+  // speed (1,041 against 1,035 TFLOP/s, interleaved).
   // With MHA (every query head its own K/V head) the CTAs working at one
   // time, spread over the row groups of all heads, touch more K/V than L2
-  // holds (the e4m3 workload read 3x its bytes).  There the units go in
-  // chunks of whole K/V heads whose K and V fit in kChunkL2Bytes, and the
-  // loads carry L2 policies (Q evict-first, K/V evict-last, O streaming):
-  // reads fell to exactly the algorithmic bytes and the e4m3 workload gained
-  // 2 % (1,482 against 1,455 TFLOP/s, interleaved).  With GQA the K/V of all
-  // heads is a quarter the size; the same changes also brought its reads to
-  // the algorithmic bytes (193 MB against 360 MB per launch) but cost 4-7 %
-  // (991 against 1,032 TFLOP/s), so GQA keeps the plain order.
+  // holds (the e4m3 workload read 3x its bytes).  There the units also go in
+  // chunks of whole K/V heads whose K and V fit in kChunkL2Bytes: reads fell
+  // to the algorithmic bytes and the e4m3 workload gained 2 % (1,482 against
+  // 1,455 TFLOP/s, interleaved).  With GQA the K/V of all heads is a quarter
+  // the size, and the chunking cost 4-7 % (991 against 1,032 TFLOP/s), so GQA
+  // keeps the plain order.
   p.chunk = p.n_pairs;
-  p.l2_hints = 0;
+  p.l2_hints = 1;
   if (p.group == 1) {
     const int lk = PAGED ? a.max_pages * kPage : a.Lk;
     const double kv_bytes = (double)lk * D * (FP8 ? 1 : 2) * 2;
     int heads = kv_bytes > 0 ? (int)(kChunkL2Bytes / kv_bytes) : p.n_pairs;
     heads = heads < 1 ? 1 : heads;
     p.chunk = heads > p.n_pairs ? p.n_pairs : heads;
-    p.l2_hints = 1;
   }
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
   cudaLaunchConfig_t cfg{};
