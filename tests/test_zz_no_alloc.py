@@ -4,8 +4,9 @@ It serves callers that cannot allocate device memory when they run decode:
 its scratch is a fixed array inside the library instead of a caller-provided
 workspace.  These GPU tests call it through the C ABI, twice in a row (the
 array keeps the first call's contents), and compare its output with the
-regular entry point's on the same inputs, within the parity tolerance used for
-decode everywhere else.  The file is named so that pytest collects it last.
+float64 oracle and with the regular entry point's on the same inputs, within
+the parity tolerance used for decode everywhere else.  The file is named so
+that pytest collects it last.
 """
 import ctypes
 
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from workloads import MQA_DECODE, DecodeShape, decode_inputs, seed_of
 
 pytestmark = pytest.mark.gpu
@@ -31,7 +33,7 @@ def _noalloc_call(cdll, d, shape, o, lse):
 
 
 @pytest.mark.parametrize("which", ["workload", "edge"])
-def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, which):
+def test_noalloc_matches_oracle_and_workspace_entry_point_on_two_calls(lib, which):
     cdll = lib.load()
     if which == "workload":
         shape = MQA_DECODE
@@ -43,6 +45,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, which):
     ref_o, ref_l = lib.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
                                          shape.scale)
     torch.cuda.synchronize()
+    o_ref, l_ref = oracle.paged_decode(kv.q, kv.k_pages, kv.v_pages, kv.block_table, kv.seq_lens, shape.scale)
+    fin_ref = np.isfinite(l_ref)
     for _ in range(2):
         o = torch.full_like(ref_o, float("nan"))
         lse = torch.full_like(ref_l, float("nan"))
@@ -55,6 +59,12 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, which):
         assert torch.equal(torch.isfinite(lse), fin)
         dl = (lse[fin].double() - ref_l[fin].double()).abs().max().item() if fin.any() else 0.0
         assert do <= O_TOL and dl <= LSE_TOL, (do, dl)
+        # against the oracle
+        on, ln = o.double().cpu().numpy(), lse.double().cpu().numpy()
+        assert np.array_equal(np.isfinite(ln), fin_ref)
+        eo = np.abs(on - o_ref).max()
+        el = np.abs(ln[fin_ref] - l_ref[fin_ref]).max() if fin_ref.any() else 0.0
+        assert eo <= O_TOL and el <= LSE_TOL, (eo, el)
 
 
 def test_noalloc_call_allocates_no_device_memory(lib):
