@@ -98,13 +98,17 @@ def test_online_recurrence_matches_brute_force(B, Hq, Hkv, Lq, Lk, D, causal, wi
 @pytest.mark.parametrize("Hq,Hkv,L,causal", [(4, 4, 33, False), (4, 4, 40, True), (8, 2, 29, True), (6, 1, 17, False)])
 def test_definition_matches_torch_sdpa(Hq, Hkv, L, causal):
     """torch's SDPA in float64 computes the same definition (its causal mask
-    is top-left aligned, identical to ours when Lq == Lk)."""
+    is top-left aligned, identical to ours when Lq == Lk).  The math backend
+    is requested explicitly: it forms softmax(scale * Q K^T) V as written, so
+    the comparison does not depend on which fused CPU kernel torch picks."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
     q = _rand((2, Hq, L, 16), 7)
     k = _rand((2, Hkv, L, 16), 8)
     v = _rand((2, Hkv, L, 16), 9)
     scale = 1 / math.sqrt(16)
-    ref = torch.nn.functional.scaled_dot_product_attention(
-        q, k, v, is_causal=causal, scale=scale, enable_gqa=(Hq != Hkv))
+    with sdpa_kernel(SDPBackend.MATH):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, k, v, is_causal=causal, scale=scale, enable_gqa=(Hq != Hkv))
     o, lse = oracle.attention(q, k, v, scale, causal)
     np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
     # LSE against torch.logsumexp over the masked score matrix
