@@ -212,6 +212,9 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Lq, int D);
  * P = exp(scale * q k^T - lse) is recomputed, rounded to bf16 for the
  * dV = P^T dO product, and dS = P * (dP - rowsum(dO * O)) to bf16 for the
  * dK and dQ products; accumulation in fp32.  Supported: bf16, D in {64, 128}.
+ * dK and dV are the same bits on every call.  dQ sums one fp32 partial per
+ * 128-key tile in whatever order the tiles finish, so it can differ between
+ * calls in the last bits of its fp32 sum (before its rounding to bf16).
  */
 ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                       const float* lse, void* dq, void* dk, void* dv,
