@@ -262,7 +262,6 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
   if (!(scale == scale) || scale <= 0.f) return ATTN_ERR_INVALID;
   if (window > 0 && !causal) return ATTN_ERR_INVALID;
-  if (causal && Lq > Lk) return ATTN_ERR_INVALID;
   if (B == 0 || Lq == 0) return ATTN_OK;
   const void* ptrs[] = {q, o, dout, dq, workspace};
   for (const void* ptr : ptrs)

@@ -207,7 +207,9 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Lq, int D);
  *   dk, dv       [B, Hkv, Lk, D] bf16 (written; each K/V head sums its group)
  *   workspace    at least attn_bwd_workspace_bytes(B, Hq, Lq, D) bytes;
  *                contents on entry do not matter
- *   scale, causal, window as attn_fwd (same mask, same alignment)
+ *   scale, causal, window as attn_fwd (same mask, same alignment); a row
+ *                that sees no key (causal with Lq > Lk) gets dQ = 0 and adds
+ *                nothing to dK, dV
  *
  * P = exp(scale * q k^T - lse) is recomputed, rounded to bf16 for the
  * dV = P^T dO product, and dS = P * (dP - rowsum(dO * O)) to bf16 for the

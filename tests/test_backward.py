@@ -6,6 +6,14 @@ would; the oracle differentiates the exact forward.  Tolerance: the products
 round P and dS to bf16 (relative 2^-9) and the outputs are bf16, so each
 gradient is compared relative to its own scale: max |err| <= 2e-2 * max |ref|
 and mean |err| <= 4e-3 * mean |ref| (about ten and two bf16 half-ulps).
+
+Rows of two keys (window 2) get a mean bound of 6e-3.  There
+dS = P (dP - Dvec) cancels to P_1 P_2 (dP_1 - dP_2), and Dvec = rowsum(dO * O)
+takes the forward's bf16 O (the stored output the recomputation uses), so O's
+rounding reaches dS without the averaging of long rows.  A float64 model of
+the kernel's three roundings (P, O and dS to bf16) gives dQ a mean error of
+4.3e-3 of its mean magnitude on that case (3.7e-3 from O alone), and the
+kernel measures the same.
 """
 import numpy as np
 import pytest
@@ -19,14 +27,14 @@ pytestmark = pytest.mark.gpu
 MAX_REL, MEAN_REL = 2e-2, 4e-3
 
 
-def _grad_check(name, got, ref):
+def _grad_check(name, got, ref, mean_rel=MEAN_REL):
     got = got.float().cpu().numpy().astype(np.float64)
     err = np.abs(got - ref)
     scale_max, scale_mean = np.abs(ref).max(), np.abs(ref).mean()
     assert np.isfinite(got).all(), f"{name}: non-finite values"
     assert err.max() <= MAX_REL * scale_max + 1e-6, f"{name}: max {err.max():.3e} vs {MAX_REL * scale_max:.3e}"
-    assert err.mean() <= MEAN_REL * scale_mean + 1e-7, f"{name}: mean {err.mean():.3e} vs {MEAN_REL * scale_mean:.3e}"
-    return err.max() / scale_max, err.mean() / scale_mean
+    assert err.mean() <= mean_rel * scale_mean + 1e-7, f"{name}: mean {err.mean():.3e} vs {mean_rel * scale_mean:.3e}"
+    return err.max() / max(scale_max, 1e-30), err.mean() / max(scale_mean, 1e-30)  # (a single key: dQ = dK = 0)
 
 
 def _case(lib, B, Hq, Hkv, Lq, Lk, D, causal, window, seed):
@@ -41,7 +49,8 @@ def _case(lib, B, Hq, Hkv, Lq, Lk, D, causal, window, seed):
     assert lib.attn_last_device_error() == 0
     o_ref, l_ref = oracle.attention(q, k, v, shape.scale, causal, window)
     dq_r, dk_r, dv_r = oracle.attention_backward(q, k, v, o_ref, do, l_ref, shape.scale, causal, window)
-    return [_grad_check(n, a, r) for n, a, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r))]
+    mean_rel = 6e-3 if 0 < window <= 2 else MEAN_REL  # rows of two keys (module docstring)
+    return [_grad_check(n, a, r, mean_rel) for n, a, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r))]
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,window", [
@@ -51,6 +60,11 @@ def _case(lib, B, Hq, Hkv, Lq, Lk, D, causal, window, seed):
     (1, 4, 1, 130, 400, 64, True, 0),       # MQA, Lq < Lk (bottom-right causal)
     (1, 4, 2, 700, 700, 128, True, 200),    # sliding window
     (1, 6, 2, 257, 257, 128, False, 0),     # group of 3, non-causal
+    (1, 2, 2, 300, 100, 128, True, 0),      # Lq > Lk: the first 200 rows see no key (their dQ is 0)
+    (1, 4, 2, 1, 1, 128, True, 0),          # a single token
+    (1, 2, 1, 17, 17, 64, True, 0),         # one ragged tile
+    (1, 4, 2, 600, 600, 64, True, 2),       # rows of two keys
+    (2, 4, 4, 129, 129, 128, False, 0),     # one row past a tile
 ])
 def test_backward_parity(lib, B, Hq, Hkv, Lq, Lk, D, causal, window):
     _case(lib, B, Hq, Hkv, Lq, Lk, D, causal, window, 500 + Lq + Hq)

@@ -166,6 +166,8 @@ FP8_SWEEP = [
     (1, 4, 4, 100, 900, True, 0),       # Lq < Lk: every row sees > 800 keys
     (1, 2, 2, 300, 100, True, 0),       # Lq > Lk: first rows see no key
     (2, 2, 1, 77, 200, False, 0),       # non-causal, short key range
+    (1, 8, 1, 600, 600, True, 0),       # MQA, group 8
+    (1, 2, 2, 17, 17, True, 0),         # one ragged tile
 ]
 
 
