@@ -58,6 +58,13 @@ constexpr uint32_t kTmS0 = 0, kTmS1 = kBlkTok, kTmO = 2 * kBlkTok;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The split kernel sees only rows of >= kShortKeys keys (shorter ones are the
+// combine kernel's), where normalising o by the exact fp32 row sum is off by
+// ~2^-9 / sqrt(n) of the weights' rounding: the sum of the rounded P, which
+// costs three instructions per key pair, is kept only with ATTN_DEC_RSUM=1.
+#ifndef ATTN_DEC_RSUM
+#define ATTN_DEC_RSUM 0
+#endif
 constexpr int kSmemPerSm = 233472;  // shared memory of an SM, 1 KB of it reserved per CTA
 // Sequences whose first query token sees fewer than kShortKeys cached tokens
 // ("short") take no part in the split kernel's page partition: the combine
@@ -819,7 +826,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           rs2[q2 & 3] = add2(rs2[q2 & 3], f2(p0, p1));
           const uint32_t bb = pack_bf16x2(p0, p1);
           pk[q2] = bb;
-          rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(bb << 16), __uint_as_float(bb & 0xFFFF0000u)));
+          if (ATTN_DEC_RSUM)
+            rr2[q2 & 3] = add2(rr2[q2 & 3], f2(__uint_as_float(bb << 16), __uint_as_float(bb & 0xFFFF0000u)));
         }
         {
           const uint64_t a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
@@ -860,7 +868,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0 && !in_range) atomicExch(p.status, kErrBounds);
       const bool write = r < p.rows && in_range;
       const size_t rec = (((size_t)b * p.Hq + kvh * p.group) * p.q_len + r) * p.max_segs + sidx;
-      const float inv = l_rnd > 0.f ? 1.f / l_rnd : 0.f;
+      const float l_o = ATTN_DEC_RSUM ? l_rnd : l_run;  // normalises o
+      const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
 #pragma unroll 1
       for (int c4 = 0; c4 < DV / 32; ++c4) {
         uint32_t raw[32];
