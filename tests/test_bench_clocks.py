@@ -51,3 +51,20 @@ def test_nvml_sampler_flags_thermal_slowdown(monkeypatch):
     c.end()
     out = c.stop()
     assert out["reasons"] == ["hw_thermal_slowdown", "sw_thermal_slowdown"]
+
+
+def test_profiled_traffic_only_for_the_captured_sources(monkeypatch):
+    """A stored ncu traffic figure is reported only while the kernel sources
+    hash to the value it was captured on; any edit turns it into None."""
+    import hashlib
+    import os
+    files = ["csrc/decode_paged.cu", "csrc/sm100_ptx.cuh"]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(bench.ROOT, "attention_flash_attn_02_b200", f), "rb") as fh:
+            h.update(fh.read())
+    current = h.hexdigest()[:16]
+    monkeypatch.setitem(bench.PROFILED_TRAFFIC, "probe", {"files": files, "sha": current, "bytes": 1234})
+    assert bench.profiled_traffic("probe") == 1234
+    monkeypatch.setitem(bench.PROFILED_TRAFFIC, "probe", {"files": files, "sha": "0" * 16, "bytes": 1234})
+    assert bench.profiled_traffic("probe") is None
